@@ -1,0 +1,161 @@
+/*
+ * vsa.h -- C ABI of libvsa.so: the forward pass of VSA-style cube-based
+ * hierarchical sparse attention on one NVIDIA B200 (sm_100a).
+ *
+ * The method (sources are web pages about it, cited by title and section):
+ *   "Faster Video Diffusion with Trainable Sparse Attention", "Approach":
+ *     mean-pool tokens into 4x4x4 cubes, run a coarse cube-to-cube dense
+ *     attention that outputs a coarse context and selects the top-K critical
+ *     cubes per query cube, run block-sparse token-level fine attention only
+ *     over the selected cubes, and combine both outputs through gates; each
+ *     cube maps to one GPU tile.
+ *   same page, "Limitations": the cube size is fixed at (4,4,4), so T, H and
+ *     W must be multiples of 4.
+ *   "Improving Video Sparse Attention with Fine-grained Router and Sparse
+ *     Rebasing", "Abstract (arXiv)": each query may attend to a variable
+ *     number of key-value blocks (read here as a top-p rule, see topk/top_p).
+ *
+ * Conventions used by every entry point
+ *   Tensors are dense, row-major, on the current CUDA device:
+ *     q, k, v, out     [B, heads, N, D]   bfloat16   (N = T*H*W, raster order
+ *                                          n = (t*H + h)*W + w)
+ *     gate_c, gate_f   [B, heads, N]      float32    (one scalar per token and
+ *                                          head; used as given)
+ *     idx              [B, heads, C, Kcap] int32     (C = N/64; selected KV
+ *                                          cube ids per query cube, ascending,
+ *                                          padded with -1)
+ *     cnt              [B, heads, C]      int32      (number of valid ids)
+ *   Cube numbering: cube c = ((t/4)*(H/4) + h/4)*(W/4) + w/4; the 64 tokens
+ *   of a cube are ordered ((t%4)*4 + h%4)*4 + w%4.
+ *   Scores use scale 1/sqrt(D). Ties in the coarse score go to the lower
+ *   cube id.
+ *   All pointers are owned by the caller; the library never frees them.
+ *   Every pointer argument must be 16-byte aligned.
+ *   Calls only enqueue work on `stream` (a cudaStream_t passed as void*; NULL
+ *   is the legacy default stream) and return without synchronising, except
+ *   vsa_check. Host-side argument errors are reported synchronously and no
+ *   work is enqueued. A failed kernel launch returns VSA_ERR_CUDA. Errors
+ *   detected on the device (a bounded wait that gave up) are recorded in the
+ *   plan's workspace and returned by the next vsa_check.
+ *   A plan must not be used by two streams at the same time.
+ */
+#ifndef VSA_H_
+#define VSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  VSA_OK = 0,
+  VSA_ERR_INVALID_ARG = 1, /* null pointer, bad count, bad mode parameters   */
+  VSA_ERR_SHAPE = 2,       /* T, H or W not a multiple of 4; B or heads < 1  */
+  VSA_ERR_UNSUPPORTED = 3, /* D not in {64, 128}; C or Kcap beyond limits    */
+  VSA_ERR_ALIGN = 4,       /* a pointer is not 16-byte aligned               */
+  VSA_ERR_CUDA = 5,        /* a CUDA call or kernel launch failed            */
+  VSA_ERR_TIMEOUT = 6,     /* a device-side wait gave up (see vsa_check)     */
+  VSA_ERR_DEVICE = 7       /* the device is not an sm_100 part               */
+} vsa_status;
+
+/* Problem description.
+ *   topk > 0 : fixed top-K mode, 1 <= topk <= C, Kcap = topk.
+ *   topk == 0: top-p mode. For query cube i, rank the KV cubes by coarse
+ *              score and keep the shortest prefix whose coarse softmax mass
+ *              reaches top_p (inclusive; all C if none does), then clamp the
+ *              count to [kmin, kmax]. 0 < top_p <= 1, 1 <= kmin <= kmax <= C,
+ *              Kcap = kmax.
+ * Limits: D in {64, 128}; C <= 4096; Kcap <= C. */
+typedef struct {
+  int B, heads, T, H, W, D;
+  int topk;
+  float top_p;
+  int kmin, kmax;
+} vsa_config;
+
+typedef struct vsa_plan_s* vsa_plan_t;
+
+/* Byte offsets of the plan's workspace regions (for inspection by tests and
+ * tools). All are relative to the workspace base passed to vsa_plan. */
+typedef struct {
+  size_t q_cube, k_cube, v_cube; /* [B*heads, C, 64, D] bf16, cube-major copies  */
+  size_t q_pool, k_pool, v_pool; /* [B*heads, C, D] fp32 cube means               */
+  size_t o_coarse;               /* [B*heads, C, D] fp32 coarse output            */
+  size_t s_coarse;               /* [B*heads, C, C] fp32 coarse scores, overwritten
+                                    by the coarse softmax probabilities           */
+  size_t cnt;                    /* [B*heads, C] int32 counts used by the fine step */
+  size_t err;                    /* int32 device error word                        */
+  size_t total;                  /* == vsa_workspace_bytes                          */
+} vsa_workspace_layout_t;
+
+/* Workspace size in bytes for cfg, or 0 if cfg is invalid. */
+size_t vsa_workspace_bytes(const vsa_config* cfg);
+
+/* Fills *layout for cfg. Returns VSA_OK or the validation error of cfg. */
+vsa_status vsa_workspace_layout(const vsa_config* cfg, vsa_workspace_layout_t* layout);
+
+/* Validates cfg and builds a plan over a caller-provided device workspace of
+ * at least vsa_workspace_bytes(cfg) bytes (256-byte aligned). The plan keeps
+ * the tensor-map descriptors of the workspace; it allocates host memory only.
+ * The workspace must stay valid until vsa_plan_destroy. */
+vsa_status vsa_plan(vsa_plan_t* out, const vsa_config* cfg, void* workspace, size_t ws_bytes);
+
+/* Whole forward pass: cube gather + mean pool, coarse attention + selection,
+ * block-sparse fine attention + gated combine.
+ *   out: [B,heads,N,D] bf16; idx: [B,heads,C,Kcap] int32 (written);
+ *   cnt: [B,heads,C] int32 (written) or NULL. */
+vsa_status vsa_run(vsa_plan_t plan, const void* q, const void* k, const void* v, const float* gate_c,
+                   const float* gate_f, void* out, int32_t* idx, int32_t* cnt, void* stream);
+
+/* Forward pass on a caller-supplied selection (the selection step is not run).
+ *   idx_in: [B,heads,C,Kcap] ascending cube ids; cnt_in: [B,heads,C] or NULL
+ *   (NULL means every row holds Kcap ids).
+ *   out: gated output (bf16, may be NULL);
+ *   out_coarse: [B,heads,C,D] fp32 coarse output (may be NULL);
+ *   out_fine:   [B,heads,N,D] fp32 fine-attention output before gating
+ *               (may be NULL). */
+vsa_status vsa_run_fixed_idx(vsa_plan_t plan, const void* q, const void* k, const void* v, const float* gate_c,
+                             const float* gate_f, const int32_t* idx_in, const int32_t* cnt_in, void* out,
+                             float* out_coarse, float* out_fine, void* stream);
+
+/* One-call form. Keeps a library-owned plan and workspace per distinct
+ * configuration (the first call for a configuration allocates device memory
+ * with cudaMalloc; later calls allocate nothing). topk > 0 selects top-K;
+ * topk == 0 selects top-p with kmin = 4 and kmax = min(128, C). */
+vsa_status vsa_forward(const void* q, const void* k, const void* v, const float* gate_c, const float* gate_f,
+                       int B, int heads, int T, int H, int W, int D, int topk, float top_p, void* out, int32_t* idx,
+                       void* stream);
+
+/* Synchronises the stream the plan last ran on, then reports (and clears) the
+ * device error word: VSA_OK; VSA_ERR_TIMEOUT if a device wait gave up;
+ * VSA_ERR_INVALID_ARG if vsa_run_fixed_idx was given a cube id outside [0, C)
+ * or a count outside [1, Kcap] (the kernel substituted cube 0 / clamped the
+ * count instead of reading out of bounds); VSA_ERR_CUDA if the stream
+ * reported an error. */
+vsa_status vsa_check(vsa_plan_t plan);
+
+/* Releases the plan (host memory only; the workspace stays the caller's). */
+void vsa_plan_destroy(vsa_plan_t plan);
+
+/* Static, human-readable name of a status code. */
+const char* vsa_status_string(vsa_status s);
+
+/* Device-side wait limit in nanoseconds used by later launches of this plan
+ * (default 1e9, minimum 1e5). Every wait of a kernel on an mbarrier gives
+ * up after this long, records VSA_ERR_TIMEOUT in the workspace error word,
+ * drains the copies and tensor-core operations it already issued, and
+ * returns. */
+vsa_status vsa_set_wait_limit_ns(vsa_plan_t plan, uint64_t limit_ns);
+
+/* Test hook for the timeout path. When `on` is nonzero, the fine-attention
+ * kernel's tensor-core issuer first waits on a barrier that nothing ever
+ * signals, so that wait runs out after the plan's wait limit and the run
+ * ends with VSA_ERR_TIMEOUT (reported by vsa_check) instead of hanging. */
+vsa_status vsa_set_debug_stall(vsa_plan_t plan, int on);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* VSA_H_ */

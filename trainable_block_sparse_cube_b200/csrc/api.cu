@@ -1,0 +1,340 @@
+// Host side of the C ABI declared in include/vsa.h: validation, workspace
+// layout, plan (tensor-map descriptors), launches and error reporting.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <new>
+
+#include "../../include/vsa.h"
+#include "vsa_common.cuh"
+
+struct vsa_plan_s {
+  vsa_config cfg;
+  int BH, N, C, kcap;
+  char* ws;
+  vsa_workspace_layout_t lay;
+  CUtensorMap tm_q, tm_k, tm_v;
+  int num_sms;
+  cudaStream_t last_stream;
+  uint64_t wait_ns;
+  int debug_stall;
+};
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+constexpr int kMaxC = 4096;
+constexpr int kMaxTopPKmax = 1024;
+
+vsa_status validate(const vsa_config* c) {
+  if (!c) return VSA_ERR_INVALID_ARG;
+  if (c->B < 1 || c->heads < 1 || c->T < 4 || c->H < 4 || c->W < 4) return VSA_ERR_SHAPE;
+  if (c->T % 4 || c->H % 4 || c->W % 4) return VSA_ERR_SHAPE;
+  if (c->D != 64 && c->D != 128) return VSA_ERR_UNSUPPORTED;
+  const long long N = (long long)c->T * c->H * c->W;
+  const long long C = N / 64;
+  if (C > kMaxC) return VSA_ERR_UNSUPPORTED;
+  if ((long long)c->B * c->heads * N * c->D >= (1LL << 40)) return VSA_ERR_UNSUPPORTED;
+  if ((long long)c->B * c->heads > 65535) return VSA_ERR_UNSUPPORTED;
+  if (c->topk < 0) return VSA_ERR_INVALID_ARG;
+  if (c->topk > 0) {
+    if (c->topk > C) return VSA_ERR_INVALID_ARG;
+  } else {
+    if (!(c->top_p > 0.f && c->top_p <= 1.f)) return VSA_ERR_INVALID_ARG;
+    if (c->kmin < 1 || c->kmin > c->kmax || c->kmax > C) return VSA_ERR_INVALID_ARG;
+    if (c->kmax > kMaxTopPKmax) return VSA_ERR_UNSUPPORTED;
+  }
+  return VSA_OK;
+}
+
+void make_layout(const vsa_config* c, vsa_workspace_layout_t* L) {
+  const size_t BH = (size_t)c->B * c->heads, N = (size_t)c->T * c->H * c->W, C = N / 64, D = c->D;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 1024);
+    return o;
+  };
+  L->q_cube = take(BH * N * D * 2);
+  L->k_cube = take(BH * N * D * 2);
+  L->v_cube = take(BH * N * D * 2);
+  L->q_pool = take(BH * C * D * 4);
+  L->k_pool = take(BH * C * D * 4);
+  L->v_pool = take(BH * C * D * 4);
+  L->o_coarse = take(BH * C * D * 4);
+  L->s_coarse = take(BH * C * C * 4);
+  L->cnt = take(BH * C * 4);
+  L->err = take(16);
+  L->total = off;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+vsa_status encode_map(CUtensorMap* m, void* base, size_t rows, int D) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return VSA_ERR_CUDA;
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? VSA_OK : VSA_ERR_CUDA;
+}
+
+vsa_status run_common(vsa_plan_t P, const void* q, const void* k, const void* v, const float* gate_c,
+                      const float* gate_f, bool select, const int32_t* idx_in, const int32_t* cnt_in, int32_t* idx_out,
+                      int32_t* cnt_out, void* out, float* out_coarse, float* out_fine, void* stream) {
+  if (!P || !q || !k || !v || !gate_c || !gate_f) return VSA_ERR_INVALID_ARG;
+  if (select && !idx_out) return VSA_ERR_INVALID_ARG;
+  if (!select && !idx_in) return VSA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, gate_c, gate_f, idx_in, cnt_in, idx_out, cnt_out, out, out_coarse, out_fine};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return VSA_ERR_ALIGN;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  P->last_stream = st;
+  const vsa_config& c = P->cfg;
+  char* ws = P->ws;
+  const vsa_workspace_layout_t& L = P->lay;
+
+  vsa::GatherParams gp{};
+  gp.src[0] = static_cast<const __nv_bfloat16*>(q);
+  gp.src[1] = static_cast<const __nv_bfloat16*>(k);
+  gp.src[2] = static_cast<const __nv_bfloat16*>(v);
+  gp.dst[0] = reinterpret_cast<__nv_bfloat16*>(ws + L.q_cube);
+  gp.dst[1] = reinterpret_cast<__nv_bfloat16*>(ws + L.k_cube);
+  gp.dst[2] = reinterpret_cast<__nv_bfloat16*>(ws + L.v_cube);
+  gp.pool[0] = reinterpret_cast<float*>(ws + L.q_pool);
+  gp.pool[1] = reinterpret_cast<float*>(ws + L.k_pool);
+  gp.pool[2] = reinterpret_cast<float*>(ws + L.v_pool);
+  gp.BH = P->BH; gp.C = P->C; gp.H = c.H; gp.W = c.W; gp.N = P->N;
+  if (vsa::launch_gather(gp, c.D, st) != cudaSuccess) return VSA_ERR_CUDA;
+
+  vsa::CoarseParams cp{};
+  cp.qpool = gp.pool[0]; cp.kpool = gp.pool[1]; cp.vpool = gp.pool[2];
+  cp.s = reinterpret_cast<float*>(ws + L.s_coarse);
+  cp.oc = reinterpret_cast<float*>(ws + L.o_coarse);
+  cp.oc_copy = out_coarse;
+  cp.idx = idx_out;
+  cp.cnt = reinterpret_cast<int32_t*>(ws + L.cnt);
+  cp.BH = P->BH; cp.C = P->C; cp.D = c.D; cp.kcap = P->kcap;
+  cp.topk = c.topk; cp.top_p = c.top_p; cp.kmin = c.kmin; cp.kmax = c.kmax;
+  cp.do_select = select ? 1 : 0;
+  cp.scale = 1.0f / std::sqrt((float)c.D);
+  if (vsa::launch_coarse(cp, st) != cudaSuccess) return VSA_ERR_CUDA;
+
+  vsa::FineParams fp{};
+  fp.tm_q = P->tm_q; fp.tm_k = P->tm_k; fp.tm_v = P->tm_v;
+  fp.idx = select ? idx_out : idx_in;
+  fp.cnt = select ? cp.cnt : cnt_in;
+  fp.oc = cp.oc;
+  fp.gate_c = gate_c; fp.gate_f = gate_f;
+  fp.out = static_cast<__nv_bfloat16*>(out);
+  fp.out_fine = out_fine;
+  fp.err = reinterpret_cast<int*>(ws + L.err);
+  fp.wait_ns = P->wait_ns;
+  fp.BH = P->BH; fp.C = P->C; fp.H = c.H; fp.W = c.W; fp.N = P->N;
+  fp.kcap = P->kcap; fp.n_items = P->BH * P->C;
+  fp.scale_log2 = 1.4426950408889634f / std::sqrt((float)c.D);
+  fp.debug_stall = P->debug_stall;
+  const int grid = fp.n_items < P->num_sms ? fp.n_items : P->num_sms;
+  if (vsa::launch_fine(fp, c.D, grid, st) != cudaSuccess) return VSA_ERR_CUDA;
+
+  if (select && cnt_out) {
+    if (cudaMemcpyAsync(cnt_out, cp.cnt, (size_t)P->BH * P->C * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return VSA_ERR_CUDA;
+  }
+  return VSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t vsa_workspace_bytes(const vsa_config* cfg) {
+  if (validate(cfg) != VSA_OK) return 0;
+  vsa_workspace_layout_t L;
+  make_layout(cfg, &L);
+  return L.total;
+}
+
+vsa_status vsa_workspace_layout(const vsa_config* cfg, vsa_workspace_layout_t* layout) {
+  if (!layout) return VSA_ERR_INVALID_ARG;
+  const vsa_status s = validate(cfg);
+  if (s != VSA_OK) return s;
+  make_layout(cfg, layout);
+  return VSA_OK;
+}
+
+vsa_status vsa_plan(vsa_plan_t* out, const vsa_config* cfg, void* workspace, size_t ws_bytes) {
+  if (!out) return VSA_ERR_INVALID_ARG;
+  *out = nullptr;
+  const vsa_status s = validate(cfg);
+  if (s != VSA_OK) return s;
+  if (!workspace) return VSA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return VSA_ERR_ALIGN;
+  vsa_workspace_layout_t L;
+  make_layout(cfg, &L);
+  if (ws_bytes < L.total) return VSA_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return VSA_ERR_CUDA;
+  int major = 0, sms = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return VSA_ERR_CUDA;
+  if (major != 10) return VSA_ERR_DEVICE;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return VSA_ERR_CUDA;
+  vsa_plan_s* P = new (std::nothrow) vsa_plan_s();
+  if (!P) return VSA_ERR_INVALID_ARG;
+  P->cfg = *cfg;
+  P->N = cfg->T * cfg->H * cfg->W;
+  P->C = P->N / 64;
+  P->BH = cfg->B * cfg->heads;
+  P->kcap = cfg->topk > 0 ? cfg->topk : cfg->kmax;
+  P->ws = static_cast<char*>(workspace);
+  P->lay = L;
+  P->num_sms = sms;
+  P->last_stream = nullptr;
+  P->wait_ns = 1000000000ull;
+  P->debug_stall = 0;
+  const size_t rows = (size_t)P->BH * P->N;
+  vsa_status e = encode_map(&P->tm_q, P->ws + L.q_cube, rows, cfg->D);
+  if (e == VSA_OK) e = encode_map(&P->tm_k, P->ws + L.k_cube, rows, cfg->D);
+  if (e == VSA_OK) e = encode_map(&P->tm_v, P->ws + L.v_cube, rows, cfg->D);
+  if (e == VSA_OK && cudaMemset(P->ws + L.err, 0, 16) != cudaSuccess) e = VSA_ERR_CUDA;
+  if (e != VSA_OK) {
+    delete P;
+    return e;
+  }
+  *out = P;
+  return VSA_OK;
+}
+
+vsa_status vsa_run(vsa_plan_t plan, const void* q, const void* k, const void* v, const float* gate_c,
+                   const float* gate_f, void* out, int32_t* idx, int32_t* cnt, void* stream) {
+  if (!out) return VSA_ERR_INVALID_ARG;
+  return run_common(plan, q, k, v, gate_c, gate_f, true, nullptr, nullptr, idx, cnt, out, nullptr, nullptr, stream);
+}
+
+vsa_status vsa_run_fixed_idx(vsa_plan_t plan, const void* q, const void* k, const void* v, const float* gate_c,
+                             const float* gate_f, const int32_t* idx_in, const int32_t* cnt_in, void* out,
+                             float* out_coarse, float* out_fine, void* stream) {
+  return run_common(plan, q, k, v, gate_c, gate_f, false, idx_in, cnt_in, nullptr, nullptr, out, out_coarse, out_fine,
+                    stream);
+}
+
+namespace {
+struct CachedPlan {
+  vsa_config cfg;
+  int device;
+  void* ws;
+  vsa_plan_t plan;
+};
+constexpr int kCacheSize = 16;
+CachedPlan g_cache[kCacheSize];
+int g_cache_n = 0;
+std::mutex g_cache_mu;
+
+bool same_cfg(const vsa_config& a, const vsa_config& b) {
+  return a.B == b.B && a.heads == b.heads && a.T == b.T && a.H == b.H && a.W == b.W && a.D == b.D &&
+         a.topk == b.topk && a.top_p == b.top_p && a.kmin == b.kmin && a.kmax == b.kmax;
+}
+}  // namespace
+
+vsa_status vsa_forward(const void* q, const void* k, const void* v, const float* gate_c, const float* gate_f, int B,
+                       int heads, int T, int H, int W, int D, int topk, float top_p, void* out, int32_t* idx,
+                       void* stream) {
+  vsa_config cfg{B, heads, T, H, W, D, topk, top_p, 0, 0};
+  if (topk == 0) {
+    const int C = (T * H * W) / 64;
+    cfg.kmax = C < 128 ? C : 128;
+    cfg.kmin = cfg.kmax < 4 ? cfg.kmax : 4;
+  }
+  const vsa_status s = validate(&cfg);
+  if (s != VSA_OK) return s;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return VSA_ERR_CUDA;
+  vsa_plan_t plan = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_cache_mu);
+    for (int i = 0; i < g_cache_n; ++i)
+      if (g_cache[i].device == dev && same_cfg(g_cache[i].cfg, cfg)) plan = g_cache[i].plan;
+    if (!plan) {
+      if (g_cache_n == kCacheSize) return VSA_ERR_UNSUPPORTED;
+      const size_t bytes = vsa_workspace_bytes(&cfg);
+      void* ws = nullptr;
+      if (cudaMalloc(&ws, bytes) != cudaSuccess) return VSA_ERR_CUDA;
+      const vsa_status ps = vsa_plan(&plan, &cfg, ws, bytes);
+      if (ps != VSA_OK) {
+        cudaFree(ws);
+        return ps;
+      }
+      g_cache[g_cache_n++] = CachedPlan{cfg, dev, ws, plan};
+    }
+  }
+  return vsa_run(plan, q, k, v, gate_c, gate_f, out, idx, nullptr, stream);
+}
+
+vsa_status vsa_check(vsa_plan_t plan) {
+  if (!plan) return VSA_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(plan->last_stream) != cudaSuccess) return VSA_ERR_CUDA;
+  int err = 0;
+  int* dev_err = reinterpret_cast<int*>(plan->ws + plan->lay.err);
+  if (cudaMemcpy(&err, dev_err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return VSA_ERR_CUDA;
+  if (err) {
+    if (cudaMemset(dev_err, 0, sizeof(int)) != cudaSuccess) return VSA_ERR_CUDA;
+  }
+  if (err & vsa::kErrTimeout) return VSA_ERR_TIMEOUT;
+  if (err & vsa::kErrBadIndex) return VSA_ERR_INVALID_ARG;
+  return VSA_OK;
+}
+
+void vsa_plan_destroy(vsa_plan_t plan) { delete plan; }
+
+const char* vsa_status_string(vsa_status s) {
+  switch (s) {
+    case VSA_OK: return "VSA_OK";
+    case VSA_ERR_INVALID_ARG: return "VSA_ERR_INVALID_ARG";
+    case VSA_ERR_SHAPE: return "VSA_ERR_SHAPE";
+    case VSA_ERR_UNSUPPORTED: return "VSA_ERR_UNSUPPORTED";
+    case VSA_ERR_ALIGN: return "VSA_ERR_ALIGN";
+    case VSA_ERR_CUDA: return "VSA_ERR_CUDA";
+    case VSA_ERR_TIMEOUT: return "VSA_ERR_TIMEOUT";
+    case VSA_ERR_DEVICE: return "VSA_ERR_DEVICE";
+  }
+  return "VSA_ERR_UNKNOWN";
+}
+
+vsa_status vsa_set_wait_limit_ns(vsa_plan_t plan, uint64_t limit_ns) {
+  if (!plan || limit_ns < 100000ull) return VSA_ERR_INVALID_ARG;
+  plan->wait_ns = limit_ns;
+  return VSA_OK;
+}
+
+vsa_status vsa_set_debug_stall(vsa_plan_t plan, int on) {
+  if (!plan) return VSA_ERR_INVALID_ARG;
+  plan->debug_stall = on ? 1 : 0;
+  return VSA_OK;
+}
+
+}  // extern "C"

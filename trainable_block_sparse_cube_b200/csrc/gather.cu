@@ -1,0 +1,80 @@
+// Cube gather and mean pool.
+//
+// "Faster Video Diffusion with Trainable Sparse Attention", "Approach":
+// tokens are grouped into 4x4x4 cubes (one GPU tile per cube) and each cube
+// is mean-pooled to one coarse token. This kernel does both in one pass over
+// q, k and v: it copies each cube's 64 raster rows into one contiguous
+// 64 x D block of the cube-major workspace (bit copy) and writes the fp32
+// mean of the 64 rows.
+//
+// One warp per (tensor, head, cube). A raster row of D bf16 is D*2 bytes; a
+// lane moves 16 bytes, so D/8 lanes cover a row and a warp covers 32/(D/8)
+// rows per step. Four consecutive w positions of a cube are contiguous in the
+// raster layout (4*D*2 bytes), and every read and write is a full 16-byte
+// vector. The pool sums are kept per lane in fp32 and combined with shuffles.
+#include "vsa_common.cuh"
+
+namespace vsa {
+
+template <int D>
+__global__ void __launch_bounds__(256) gather_pool_kernel(const GatherParams p) {
+  constexpr int LPR = D / 8;        // lanes per row
+  constexpr int RPS = 32 / LPR;     // rows per warp step
+  constexpr int STEPS = kCube / RPS;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = blockIdx.x * 8 + warp;
+  const int bh = blockIdx.y, tensor = blockIdx.z;
+  if (c >= p.C) return;
+  const int sub = lane / LPR, chunk = lane % LPR;
+  const __nv_bfloat16* src = p.src[tensor] + (size_t)bh * p.N * D + chunk * 8;
+  __nv_bfloat16* dst = p.dst[tensor] + ((size_t)bh * p.C + c) * kCube * D + chunk * 8;
+
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+
+  constexpr int U = STEPS < 8 ? STEPS : 8;
+#pragma unroll
+  for (int s0 = 0; s0 < STEPS; s0 += U) {
+    int4 v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int r = (s0 + u) * RPS + sub;
+      const int n = cube_token(c, r, p.H, p.W);
+      v[u] = __ldg(reinterpret_cast<const int4*>(src + (size_t)n * D));
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int r = (s0 + u) * RPS + sub;
+      *reinterpret_cast<int4*>(dst + (size_t)r * D) = v[u];
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(h2[e]);
+        acc[2 * e] += f.x;
+        acc[2 * e + 1] += f.y;
+      }
+    }
+  }
+#pragma unroll
+  for (int off = LPR; off < 32; off <<= 1)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+  if (sub == 0) {
+    float* pool = p.pool[tensor] + ((size_t)bh * p.C + c) * D + chunk * 8;
+    const float inv = 1.0f / kCube;
+    *reinterpret_cast<float4*>(pool) = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+    *reinterpret_cast<float4*>(pool + 4) = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+  }
+}
+
+cudaError_t launch_gather(const GatherParams& p, int D, cudaStream_t st) {
+  dim3 grid((p.C + 7) / 8, p.BH, 3);
+  if (D == 128)
+    gather_pool_kernel<128><<<grid, 256, 0, st>>>(p);
+  else
+    gather_pool_kernel<64><<<grid, 256, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace vsa

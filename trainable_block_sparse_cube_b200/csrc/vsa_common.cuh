@@ -1,0 +1,68 @@
+// Shared definitions of the VSA kernels (device side) and their launchers.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace vsa {
+
+// Bits of the device error word kept in the workspace.
+enum : int { kErrTimeout = 1, kErrBadIndex = 2 };
+
+constexpr int kCube = 64;  // tokens per 4x4x4 cube
+
+// Raster token index of in-cube slot r of cube c (cube and slot numbering as
+// documented in include/vsa.h).
+__host__ __device__ __forceinline__ int cube_token(int c, int r, int H, int W) {
+  const int Hc = H >> 2, Wc = W >> 2;
+  const int ct = c / (Hc * Wc), ch = (c / Wc) % Hc, cw = c % Wc;
+  const int t = 4 * ct + (r >> 4), h = 4 * ch + ((r >> 2) & 3), w = 4 * cw + (r & 3);
+  return (t * H + h) * W + w;
+}
+
+struct GatherParams {
+  const __nv_bfloat16* src[3];  // q, k, v raster [BH, N, D]
+  __nv_bfloat16* dst[3];        // cube-major [BH, C, 64, D]
+  float* pool[3];               // [BH, C, D] cube means
+  int BH, C, H, W, N;
+};
+
+struct CoarseParams {
+  const float* qpool;  // [BH, C, D]
+  const float* kpool;
+  const float* vpool;
+  float* s;            // [BH, C, C] scores, then probabilities
+  float* oc;           // [BH, C, D]
+  float* oc_copy;      // optional second destination of oc (may be null)
+  int32_t* idx;        // [BH, C, kcap]
+  int32_t* cnt;        // [BH, C]
+  int BH, C, D, kcap;
+  int topk;            // > 0: top-K; 0: top-p
+  float top_p;
+  int kmin, kmax;
+  int do_select;       // 0: only probabilities (selection supplied by the caller)
+  float scale;         // 1/sqrt(D)
+};
+
+struct FineParams {
+  CUtensorMap tm_q, tm_k, tm_v;  // 2-D maps over the cube-major copies, rows of D bf16
+  const int32_t* idx;            // [BH, C, kcap]
+  const int32_t* cnt;            // [BH, C] or null (then every row has kcap ids)
+  const float* oc;               // [BH, C, D]
+  const float* gate_c;           // [BH, N]
+  const float* gate_f;           // [BH, N]
+  __nv_bfloat16* out;            // [BH, N, D] or null
+  float* out_fine;               // [BH, N, D] or null
+  int* err;
+  unsigned long long wait_ns;
+  int BH, C, H, W, N, kcap, n_items;
+  float scale_log2;              // log2(e)/sqrt(D)
+  int debug_stall;
+};
+
+cudaError_t launch_gather(const GatherParams& p, int D, cudaStream_t st);
+cudaError_t launch_coarse(const CoarseParams& p, cudaStream_t st);
+cudaError_t launch_fine(const FineParams& p, int D, int grid, cudaStream_t st);
+
+}  // namespace vsa
