@@ -155,6 +155,20 @@ vsa_status vsa_set_wait_limit_ns(vsa_plan_t plan, uint64_t limit_ns);
  * ends with VSA_ERR_TIMEOUT (reported by vsa_check) instead of hanging. */
 vsa_status vsa_set_debug_stall(vsa_plan_t plan, int on);
 
+/* Stage timing for benchmarks. When `on` is nonzero, later runs of this plan
+ * record CUDA events (created here, once) on the run's stream around its three
+ * stages: gather + pool, coarse attention + selection, fine attention +
+ * combine. */
+vsa_status vsa_set_stage_timing(vsa_plan_t plan, int on);
+
+/* Waits for the events of the last timed run and writes the device time of
+ * its stages in milliseconds to ms[0] (gather + pool), ms[1] (coarse),
+ * ms[2] (fine). VSA_ERR_INVALID_ARG if timing is off or nothing ran yet. */
+vsa_status vsa_stage_times(vsa_plan_t plan, float* ms);
+
+/* Number of kernel launches one vsa_run / vsa_run_fixed_idx call makes. */
+int vsa_kernels_per_run(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -22,6 +22,9 @@ struct vsa_plan_s {
   cudaStream_t last_stream;
   uint64_t wait_ns;
   int debug_stall;
+  int timing;        // record stage events
+  int timed_runs;    // runs recorded since timing was enabled
+  cudaEvent_t ev[4];
 };
 
 namespace {
@@ -130,7 +133,9 @@ vsa_status run_common(vsa_plan_t P, const void* q, const void* k, const void* v,
   gp.pool[1] = reinterpret_cast<float*>(ws + L.k_pool);
   gp.pool[2] = reinterpret_cast<float*>(ws + L.v_pool);
   gp.BH = P->BH; gp.C = P->C; gp.H = c.H; gp.W = c.W; gp.N = P->N;
+  if (P->timing && cudaEventRecord(P->ev[0], st) != cudaSuccess) return VSA_ERR_CUDA;
   if (vsa::launch_gather(gp, c.D, st) != cudaSuccess) return VSA_ERR_CUDA;
+  if (P->timing && cudaEventRecord(P->ev[1], st) != cudaSuccess) return VSA_ERR_CUDA;
 
   vsa::CoarseParams cp{};
   cp.qpool = gp.pool[0]; cp.kpool = gp.pool[1]; cp.vpool = gp.pool[2];
@@ -160,7 +165,12 @@ vsa_status run_common(vsa_plan_t P, const void* q, const void* k, const void* v,
   fp.scale_log2 = 1.4426950408889634f / std::sqrt((float)c.D);
   fp.debug_stall = P->debug_stall;
   const int grid = fp.n_items < P->num_sms ? fp.n_items : P->num_sms;
+  if (P->timing && cudaEventRecord(P->ev[2], st) != cudaSuccess) return VSA_ERR_CUDA;
   if (vsa::launch_fine(fp, c.D, grid, st) != cudaSuccess) return VSA_ERR_CUDA;
+  if (P->timing) {
+    if (cudaEventRecord(P->ev[3], st) != cudaSuccess) return VSA_ERR_CUDA;
+    P->timed_runs++;
+  }
 
   if (select && cnt_out) {
     if (cudaMemcpyAsync(cnt_out, cp.cnt, (size_t)P->BH * P->C * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
@@ -309,7 +319,12 @@ vsa_status vsa_check(vsa_plan_t plan) {
   return VSA_OK;
 }
 
-void vsa_plan_destroy(vsa_plan_t plan) { delete plan; }
+void vsa_plan_destroy(vsa_plan_t plan) {
+  if (!plan) return;
+  if (plan->ev[0])
+    for (int i = 0; i < 4; ++i) cudaEventDestroy(plan->ev[i]);
+  delete plan;
+}
 
 const char* vsa_status_string(vsa_status s) {
   switch (s) {
@@ -330,6 +345,27 @@ vsa_status vsa_set_wait_limit_ns(vsa_plan_t plan, uint64_t limit_ns) {
   plan->wait_ns = limit_ns;
   return VSA_OK;
 }
+
+vsa_status vsa_set_stage_timing(vsa_plan_t plan, int on) {
+  if (!plan) return VSA_ERR_INVALID_ARG;
+  if (on && !plan->ev[0]) {
+    for (int i = 0; i < 4; ++i)
+      if (cudaEventCreate(&plan->ev[i]) != cudaSuccess) return VSA_ERR_CUDA;
+  }
+  plan->timing = on ? 1 : 0;
+  plan->timed_runs = 0;
+  return VSA_OK;
+}
+
+vsa_status vsa_stage_times(vsa_plan_t plan, float* ms) {
+  if (!plan || !ms || !plan->timing || plan->timed_runs == 0) return VSA_ERR_INVALID_ARG;
+  if (cudaEventSynchronize(plan->ev[3]) != cudaSuccess) return VSA_ERR_CUDA;
+  for (int i = 0; i < 3; ++i)
+    if (cudaEventElapsedTime(&ms[i], plan->ev[i], plan->ev[i + 1]) != cudaSuccess) return VSA_ERR_CUDA;
+  return VSA_OK;
+}
+
+int vsa_kernels_per_run(void) { return 5; }
 
 vsa_status vsa_set_debug_stall(vsa_plan_t plan, int on) {
   if (!plan) return VSA_ERR_INVALID_ARG;

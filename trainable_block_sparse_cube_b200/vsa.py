@@ -20,7 +20,7 @@ STATUS = {0: "VSA_OK", 1: "VSA_ERR_INVALID_ARG", 2: "VSA_ERR_SHAPE", 3: "VSA_ERR
 
 EXPORTED = ["vsa_workspace_bytes", "vsa_workspace_layout", "vsa_plan", "vsa_run", "vsa_run_fixed_idx",
             "vsa_forward", "vsa_check", "vsa_plan_destroy", "vsa_status_string", "vsa_set_wait_limit_ns",
-            "vsa_set_debug_stall"]
+            "vsa_set_debug_stall", "vsa_set_stage_timing", "vsa_stage_times", "vsa_kernels_per_run"]
 
 
 class VSAError(RuntimeError):
@@ -74,6 +74,12 @@ def load():
     L.vsa_set_wait_limit_ns.restype = i32
     L.vsa_set_debug_stall.argtypes = [vp, i32]
     L.vsa_set_debug_stall.restype = i32
+    L.vsa_set_stage_timing.argtypes = [vp, i32]
+    L.vsa_set_stage_timing.restype = i32
+    L.vsa_stage_times.argtypes = [vp, ctypes.POINTER(ctypes.c_float)]
+    L.vsa_stage_times.restype = i32
+    L.vsa_kernels_per_run.argtypes = []
+    L.vsa_kernels_per_run.restype = i32
     _lib = L
     return L
 
@@ -186,6 +192,15 @@ class Plan:
 
     def set_debug_stall(self, on: bool):
         _check(load().vsa_set_debug_stall(self._h, 1 if on else 0), "vsa_set_debug_stall")
+
+    def set_stage_timing(self, on: bool):
+        _check(load().vsa_set_stage_timing(self._h, 1 if on else 0), "vsa_set_stage_timing")
+
+    def stage_times(self):
+        """Device ms of (gather+pool, coarse, fine) of the last timed run."""
+        ms = (ctypes.c_float * 3)()
+        _check(load().vsa_stage_times(self._h, ms), "vsa_stage_times")
+        return tuple(float(x) for x in ms)
 
     # ------------------------------------------------------------ workspace views
     def workspace_view(self, region: str, dtype, shape):
