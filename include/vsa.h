@@ -128,6 +128,33 @@ vsa_status vsa_forward(const void* q, const void* k, const void* v, const float*
                        int B, int heads, int T, int H, int W, int D, int topk, float top_p, void* out, int32_t* idx,
                        void* stream);
 
+/* Forward pass for callers that cannot allocate memory: for example code
+ * running under a strict memory budget, inside a custom allocator that must
+ * own every device byte, or in a real-time loop where cudaMalloc (which may
+ * synchronise the device) is not allowed. It takes the same arguments and
+ * returns the same results as vsa_forward, but allocates nothing -- no
+ * cudaMalloc, no host heap: its workspace is one fixed device array of
+ * VSA_NOALLOC_SCRATCH_BYTES inside libvsa.so, which every GPU that loads
+ * the library holds until the process exits.
+ * The pages describing the method have no counterpart of this entry point.
+ *   - Configurations whose workspace (vsa_workspace_bytes) exceeds
+ *     VSA_NOALLOC_SCRATCH_BYTES are rejected with VSA_ERR_UNSUPPORTED before
+ *     anything is enqueued.
+ *   - The first call on each device looks up the device address of the
+ *     array (cudaGetSymbolAddress); make that first call before any stream
+ *     capture starts.
+ *   - All calls share the one array: calls whose work overlaps on the GPU
+ *     (different streams, or different host threads, without ordering
+ *     between them) race on it. Serialise them, e.g. on one stream.
+ *   - The array keeps the previous call's contents; the call clears the
+ *     part that must start at zero (the device error word) itself.
+ *   - Device-side errors of this entry point are not reported (there is no
+ *     plan to query with vsa_check). */
+#define VSA_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+vsa_status vsa_forward_noalloc(const void* q, const void* k, const void* v, const float* gate_c,
+                               const float* gate_f, int B, int heads, int T, int H, int W, int D, int topk,
+                               float top_p, void* out, int32_t* idx, void* stream);
+
 /* Synchronises the stream the plan last ran on, then reports (and clears) the
  * device error word: VSA_OK; VSA_ERR_TIMEOUT if a device wait gave up;
  * VSA_ERR_INVALID_ARG if vsa_run_fixed_idx was given a cube id outside [0, C)

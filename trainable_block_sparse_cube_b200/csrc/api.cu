@@ -305,6 +305,81 @@ vsa_status vsa_forward(const void* q, const void* k, const void* v, const float*
   return vsa_run(plan, q, k, v, gate_c, gate_f, out, idx, nullptr, stream);
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free forward (vsa_forward_noalloc). The workspace is this one
+// file-scope device array; host code only ever passes its device address,
+// looked up once per device with cudaGetSymbolAddress (in host code the
+// array's name is a host-side stand-in, not a device address).
+namespace {
+static __device__ __align__(256) unsigned char g_noalloc_scratch[VSA_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kNoallocMaxDevices = 64;
+void* g_noalloc_addr[kNoallocMaxDevices];
+std::mutex g_noalloc_mu;
+
+vsa_status noalloc_scratch(int dev, void** out) {
+  if (dev < 0 || dev >= kNoallocMaxDevices) return VSA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return VSA_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return VSA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+vsa_status vsa_forward_noalloc(const void* q, const void* k, const void* v, const float* gate_c,
+                               const float* gate_f, int B, int heads, int T, int H, int W, int D, int topk,
+                               float top_p, void* out, int32_t* idx, void* stream) {
+  vsa_config cfg{B, heads, T, H, W, D, topk, top_p, 0, 0};
+  if (topk == 0) {
+    const int C = (T * H * W) / 64;
+    cfg.kmax = C < 128 ? C : 128;
+    cfg.kmin = cfg.kmax < 4 ? cfg.kmax : 4;
+  }
+  vsa_status s = validate(&cfg);
+  if (s != VSA_OK) return s;
+  if (!out || !idx) return VSA_ERR_INVALID_ARG;
+  vsa_workspace_layout_t L;
+  make_layout(&cfg, &L);
+  if (L.total > VSA_NOALLOC_SCRATCH_BYTES) return VSA_ERR_UNSUPPORTED;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return VSA_ERR_CUDA;
+  int major = 0, sms = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return VSA_ERR_CUDA;
+  if (major != 10) return VSA_ERR_DEVICE;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return VSA_ERR_CUDA;
+  void* scratch = nullptr;
+  s = noalloc_scratch(dev, &scratch);
+  if (s != VSA_OK) return s;
+  // A plan on the stack over the static workspace (no heap allocation).
+  vsa_plan_s P{};
+  P.cfg = cfg;
+  P.N = T * H * W;
+  P.C = P.N / 64;
+  P.BH = B * heads;
+  P.kcap = cfg.topk > 0 ? cfg.topk : cfg.kmax;
+  P.ws = static_cast<char*>(scratch);
+  P.lay = L;
+  P.num_sms = sms;
+  P.wait_ns = 1000000000ull;
+  const size_t rows = (size_t)P.BH * P.N;
+  s = encode_map(&P.tm_q, P.ws + L.q_cube, rows, D);
+  if (s == VSA_OK) s = encode_map(&P.tm_k, P.ws + L.k_cube, rows, D);
+  if (s == VSA_OK) s = encode_map(&P.tm_v, P.ws + L.v_cube, rows, D);
+  if (s != VSA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(P.ws + L.err, 0, 16, st) != cudaSuccess) return VSA_ERR_CUDA;
+  return run_common(&P, q, k, v, gate_c, gate_f, true, nullptr, nullptr, idx, nullptr, out, nullptr, nullptr,
+                    stream);
+}
+
 vsa_status vsa_check(vsa_plan_t plan) {
   if (!plan) return VSA_ERR_INVALID_ARG;
   if (cudaStreamSynchronize(plan->last_stream) != cudaSuccess) return VSA_ERR_CUDA;

@@ -20,7 +20,8 @@ STATUS = {0: "VSA_OK", 1: "VSA_ERR_INVALID_ARG", 2: "VSA_ERR_SHAPE", 3: "VSA_ERR
 
 EXPORTED = ["vsa_workspace_bytes", "vsa_workspace_layout", "vsa_plan", "vsa_run", "vsa_run_fixed_idx",
             "vsa_forward", "vsa_check", "vsa_plan_destroy", "vsa_status_string", "vsa_set_wait_limit_ns",
-            "vsa_set_debug_stall", "vsa_set_stage_timing", "vsa_stage_times", "vsa_kernels_per_run"]
+            "vsa_set_debug_stall", "vsa_set_stage_timing", "vsa_stage_times", "vsa_kernels_per_run",
+            "vsa_forward_noalloc"]
 
 
 class VSAError(RuntimeError):
@@ -80,6 +81,8 @@ def load():
     L.vsa_stage_times.restype = i32
     L.vsa_kernels_per_run.argtypes = []
     L.vsa_kernels_per_run.restype = i32
+    L.vsa_forward_noalloc.argtypes = [vp] * 5 + [i32] * 7 + [ctypes.c_float, vp, vp, vp]
+    L.vsa_forward_noalloc.restype = i32
     _lib = L
     return L
 
