@@ -9,27 +9,37 @@
 //
 // One work item = one query cube (64 tokens) of one (batch, head). A
 // persistent CTA per SM walks items in (batch*head)-major order so the K/V
-// cubes of one or two heads stay resident in L2.
+// cubes of one or two heads stay resident in L2. Each step covers two of the
+// item's selected KV cubes (128 keys):
+//   S[64 q x 128 keys] = Q . K_pair^T     tcgen05.mma M=64, N=128, A = Q in TMEM
+//   O[64 q x D]       += P . V_pair       tcgen05.mma M=64, N=D,   A = P in TMEM
+// Shared memory bandwidth, not the tensor core, bounds this kernel (every
+// selected KV cube is used by one query cube, so each K/V byte is written to
+// and read from shared memory once). Keeping Q and P in tensor memory leaves
+// only the K and V tiles in shared memory: 64 KB written + 64 KB read per step.
 //
-// The 64-row query tile is too short for the tensor core's 128-row M, so both
-// products are computed transposed, with two selected KV cubes (128 keys)
-// per step:
-//   S^T[128 keys x 64 q]  = K_pair[128 x D] . Q[64 x D]^T      (tcgen05, M=128, N=64)
-//   O^T[D x 64 q]        += V_pair^T[D x 128] . P^T[128 x 64]  (tcgen05, M=D,   N=64)
-// Both accumulate in tensor memory (TMEM). Each softmax thread owns one key
-// row of S^T (64 query columns); column statistics (the running max) are
-// reduced across the 128 softmax threads only when some score exceeds the
-// current reference by more than 2^8 (lazy rescaling), which after the first
-// step of an item is rare. Row sums are kept as per-thread partials and
-// reduced once per item.
+// The M=64 accumulators occupy 16 lanes of each 32-lane TMEM quarter; the
+// 16-lane tcgen05.ld/st shapes spread those lanes over all 32 threads of a
+// warp: with .16x256b a thread holds rows r and r+8 of its quarter and
+// columns {8j + 2(t%4), 8j + 2(t%4) + 1}, so four threads share a row and a
+// row max / row sum needs two shuffles. P is packed to bf16 pairs and written
+// back with .16x128b, whose column 4j + (t%4) is exactly the pair the thread
+// holds. Softmax is online per row with lazy rescaling: the reference max of a
+// row moves only when a score exceeds it by more than 2^8, which after the
+// first step of an item is rare; O is then rescaled in place.
 //
-// Warp roles (256 threads):
-//   warp 0  TMA producer for Q and K tiles (lane 0 issues)
-//   warp 1  TMA producer for V tiles (a second issuing thread doubles the
-//           TMA request rate a single thread can sustain)
-//   warp 2  TMEM allocation and the single-thread tcgen05.mma issuer
-//   warp 3  idle
-//   warps 4-7  softmax (key row = TMEM lane) and the epilogue
+// Warp roles (384 threads):
+//   warp 0      TMA producer of K tiles (3-stage ring)
+//   warp 1      TMA producer of V tiles (3-stage ring; a second issuing thread,
+//               since one thread cannot keep the L2 -> SM stream full)
+//   warp 2      TMEM allocation, single-thread tcgen05.mma issuer
+//   warp 3      idle
+//   warps 4-7   softmax (warp w reads TMEM quarter w%4)
+//   warps 8-11  epilogue: loads each item's Q into TMEM, reads O, applies
+//               1/l and the gates, writes the output rows
+// MMA order: S(g), O(g-1), S(g+1), O(g), ... over the CTA's steps. A tcgen05
+// commit covers every earlier MMA of the issuing thread, so "S(g) complete"
+// implies "O(g-2) complete", which is what makes the S/P double buffer safe.
 //
 // Every mbarrier wait is bounded (plan wait limit). A wait that gives up
 // records kErrTimeout, sets a CTA-wide abort flag that makes every later wait
@@ -44,11 +54,12 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kThreads = 256;
-constexpr int kNK = 2;  // K tile stages
-constexpr int kNV = 2;  // V tile stages
-constexpr uint32_t kTmemCols = 256;
-constexpr int kSoftmaxBar = 1;  // named barrier of the 128 softmax threads
+constexpr int kThreads = 384;
+constexpr int kKStages = 3;
+constexpr int kVStages = 3;
+constexpr uint32_t kTmemCols = 512;
+// TMEM columns: S/P buffers at 0 and 128, O at 256, Q buffers at 384 and 448.
+constexpr uint32_t kColS = 0, kColO = 256, kColQ = 384;
 
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
@@ -56,80 +67,101 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-__device__ __forceinline__ void softmax_sync() {
-  asm volatile("bar.sync %0, 128;" ::"n"(kSoftmaxBar) : "memory");
-}
-// Barrier over the 128 softmax threads that also ORs a predicate.
-__device__ __forceinline__ bool softmax_sync_or(bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred pi, po;\n\t"
-      "setp.ne.u32 pi, %1, 0;\n\t"
-      "bar.red.or.pred po, %2, 128, pi;\n\t"
-      "selp.u32 %0, 1, 0, po;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)v), "n"(kSoftmaxBar)
-      : "memory");
-  return r != 0;
-}
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
 
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+// ---- 16-lane TMEM shapes (lanes base..base+15 of the warp's quarter) ----
+#define VSA_O4(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3])
+#define VSA_I4(i) "r"(r[i]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3])
+// .16x256b.x16: 128 columns; r[4j..4j+3] = (row a: col c, c+1; row a+8: col c, c+1), c = 8j + 2(t%4).
+__device__ __forceinline__ void ld_16x256b_x16(uint32_t taddr, uint32_t (&r)[64]) {
   asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "tcgen05.ld.sync.aligned.16x256b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+      "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
+      : VSA_O4(0), VSA_O4(4), VSA_O4(8), VSA_O4(12), VSA_O4(16), VSA_O4(20), VSA_O4(24), VSA_O4(28),
+        VSA_O4(32), VSA_O4(36), VSA_O4(40), VSA_O4(44), VSA_O4(48), VSA_O4(52), VSA_O4(56), VSA_O4(60)
+      : "r"(taddr));
+}
+__device__ __forceinline__ void ld_16x256b_x8(uint32_t taddr, uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x8.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : VSA_O4(0), VSA_O4(4), VSA_O4(8), VSA_O4(12), VSA_O4(16), VSA_O4(20), VSA_O4(24), VSA_O4(28)
+      : "r"(taddr));
+}
+__device__ __forceinline__ void st_16x256b_x16(uint32_t taddr, const uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x256b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,"
+      "%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,"
+      "%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64};" ::"r"(taddr),
+      VSA_I4(0), VSA_I4(4), VSA_I4(8), VSA_I4(12), VSA_I4(16), VSA_I4(20), VSA_I4(24), VSA_I4(28), VSA_I4(32),
+      VSA_I4(36), VSA_I4(40), VSA_I4(44), VSA_I4(48), VSA_I4(52), VSA_I4(56), VSA_I4(60)
+      : "memory");
+}
+__device__ __forceinline__ void st_16x256b_x8(uint32_t taddr, const uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x256b.x8.b32 [%0], "
       "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
       "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
-      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
-      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      VSA_I4(0), VSA_I4(4), VSA_I4(8), VSA_I4(12), VSA_I4(16), VSA_I4(20), VSA_I4(24), VSA_I4(28)
       : "memory");
 }
+__device__ __forceinline__ void st_16x256b_x4(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x256b.x4.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      VSA_I4(0), VSA_I4(4), VSA_I4(8), VSA_I4(12)
+      : "memory");
+}
+// .16x128b.x16: 64 columns; r[2j] -> (row a, col 4j + t%4), r[2j+1] -> (row a+8, same col).
+__device__ __forceinline__ void st_16x128b_x16(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x128b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      VSA_I4(0), VSA_I4(4), VSA_I4(8), VSA_I4(12), VSA_I4(16), VSA_I4(20), VSA_I4(24), VSA_I4(28)
+      : "memory");
+}
+#undef VSA_O4
+#undef VSA_I4
 
-// Column-wise reduction of a 64-wide row held by each lane: after the call,
-// v[0] and v[1] hold the reduction over the 32 lanes of columns 2*lane and
-// 2*lane+1 (recursive halving: each stage keeps half the columns and
-// exchanges the other half with the partner lane).
-template <bool IS_MAX>
-__device__ __forceinline__ void warp_colreduce64(float (&v)[64], int lane) {
-#define VSA_STAGE(W, BIT)                                             \
-  {                                                                   \
-    const bool up = (lane & BIT) != 0;                                \
-    _Pragma("unroll") for (int j = 0; j < W; ++j) {                   \
-      const float send = up ? v[j] : v[j + W];                        \
-      const float keep = up ? v[j + W] : v[j];                        \
-      const float recv = __shfl_xor_sync(0xffffffffu, send, BIT);     \
-      v[j] = IS_MAX ? fmaxf(keep, recv) : keep + recv;                \
-    }                                                                 \
-  }
-  VSA_STAGE(32, 16)
-  VSA_STAGE(16, 8)
-  VSA_STAGE(8, 4)
-  VSA_STAGE(4, 2)
-  VSA_STAGE(2, 1)
-#undef VSA_STAGE
+// D[tmem] (+)= A[tmem] * B[smem]^T ; issued by a single thread.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
 
 template <int D>
 struct Layout {
   static constexpr int NH = D / 64;              // 128-byte column groups of a row
-  static constexpr int Q_BYTES = 64 * D * 2;     // one query cube
   static constexpr int KV_BYTES = 128 * D * 2;   // two KV cubes
-  static constexpr int P_BYTES = 128 * 64 * 2;   // P^T, 128 keys x 64 queries
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
-  static constexpr int OFF_V = OFF_K + kNK * KV_BYTES;
-  static constexpr int OFF_P = OFF_V + kNV * KV_BYTES;
-  static constexpr int TILE_BYTES = OFF_P + 2 * P_BYTES;
-  static constexpr int SMEM_BYTES = TILE_BYTES + 1024;  // + alignment slack
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + kKStages * KV_BYTES;
+  static constexpr int OFF_STAGE = OFF_V + kVStages * KV_BYTES;   // output staging, 64 x D bf16
+  static constexpr int TILE_BYTES = OFF_STAGE + 64 * D * 2;
+  static constexpr int SMEM_BYTES = TILE_BYTES + 1024;            // + alignment slack
 };
 
 struct __align__(8) Bars {
-  uint64_t q_full[2], q_empty[2];
-  uint64_t k_full[kNK], k_empty[kNK];
-  uint64_t v_full[kNV], v_empty[kNV];
-  uint64_t s_full[2], s_empty[2];
-  uint64_t p_full[2], p_empty[2];
-  uint64_t o_full[2], o_empty[2];
+  uint64_t k_full[kKStages], k_empty[kKStages];
+  uint64_t v_full[kVStages], v_empty[kVStages];
+  uint64_t q_full[2];      // epilogue warps -> MMA: Q of the item in TMEM (count 4)
+  uint64_t s_full[2];      // MMA -> softmax: S of a step (commit)
+  uint64_t p_full[2];      // softmax -> MMA: P of a step in TMEM (count 4)
+  uint64_t l_full[2];      // softmax -> epilogue: 1/l of an item (count 4)
+  uint64_t o_step;         // MMA: each O step completed (commit)
+  uint64_t o_full;         // MMA -> epilogue: last O step of an item (commit)
+  uint64_t o_empty;        // epilogue -> MMA: O read out (count 4)
   uint64_t drain, stall;
 };
 
@@ -137,13 +169,7 @@ struct alignas(16) Shared {
   Bars bar;
   uint32_t tmem_base;
   int abort_flag;
-  alignas(16) float m_ref[64];   // running max per query (log2 units, scaled)
-  alignas(16) float alpha[64];   // rescale factor of the last max update
-  alignas(16) float red[4][64];  // per-warp column partials
-  alignas(16) float inv_l[64];
-  alignas(16) float gc[64];
-  alignas(16) float gf[64];
-  alignas(16) int tok[64];       // raster token of each query row of the item
+  alignas(16) float inv_l[2][64];
 };
 
 struct Waiter {
@@ -185,6 +211,7 @@ __device__ __forceinline__ int item_count(const FineParams& p, int item, bool* b
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __grid_constant__ FineParams p) {
   using L = Layout<D>;
+  constexpr uint32_t kQCols = D / 2;  // Q in TMEM: bf16 pairs
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ Shared sh;
@@ -194,25 +221,23 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
   const int C = p.C;
 
   if (tid == 0) {
+    for (int i = 0; i < kKStages; ++i) { mbar_init(&B.k_full[i], 1); mbar_init(&B.k_empty[i], 1); }
+    for (int i = 0; i < kVStages; ++i) { mbar_init(&B.v_full[i], 1); mbar_init(&B.v_empty[i], 1); }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&B.q_full[i], 1);
-      mbar_init(&B.q_empty[i], 4);
+      mbar_init(&B.q_full[i], 4);
       mbar_init(&B.s_full[i], 1);
-      mbar_init(&B.s_empty[i], 4);
       mbar_init(&B.p_full[i], 4);
-      mbar_init(&B.p_empty[i], 1);
-      mbar_init(&B.o_full[i], 1);
-      mbar_init(&B.o_empty[i], 4);
+      mbar_init(&B.l_full[i], 4);
     }
-    for (int i = 0; i < kNK; ++i) { mbar_init(&B.k_full[i], 1); mbar_init(&B.k_empty[i], 1); }
-    for (int i = 0; i < kNV; ++i) { mbar_init(&B.v_full[i], 1); mbar_init(&B.v_empty[i], 1); }
+    mbar_init(&B.o_step, 1);
+    mbar_init(&B.o_full, 1);
+    mbar_init(&B.o_empty, 4);
     mbar_init(&B.drain, 1);
     mbar_init(&B.stall, 1);
     sh.abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    prefetch_tmap(&p.tm_q);
     prefetch_tmap(&p.tm_k);
     prefetch_tmap(&p.tm_v);
   }
@@ -224,39 +249,22 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
-  // TMEM columns: S^T buffers at [0,64) and [64,128); O^T buffers at [128,192) and [192,256).
-  const uint32_t tS = tmem, tO = tmem + 128;
 
   if (warp == 0 || warp == 1) {
-    // ------------------------------------------------------------ producers
+    // ------------------------------------------------------------ K / V producers
     const bool is_k = (warp == 0);
     uint64_t* full = is_k ? B.k_full : B.v_full;
     uint64_t* empty = is_k ? B.k_empty : B.v_empty;
-    constexpr int NS = kNK;  // kNK == kNV
+    constexpr int NS = kKStages;  // == kVStages
     uint8_t* ring = tiles + (is_k ? L::OFF_K : L::OFF_V);
     const CUtensorMap* tm = is_k ? &p.tm_k : &p.tm_v;
-    int g = 0;                       // tiles issued
-    int last_q = -1;                 // last item whose Q load was issued
     bool bad = false, aborted = false;
-    for (int li = 0, item = blockIdx.x; item < p.n_items && !aborted; ++li, item += gridDim.x) {
+    int g = 0;  // steps issued
+    for (int item = blockIdx.x; item < p.n_items && !aborted; item += gridDim.x) {
       const int bh = item / C;
       const int n = item_count(p, item, &bad);
       const int ntiles = (n + 1) >> 1;
       const int32_t* list = p.idx + (size_t)item * p.kcap;
-      if (is_k) {
-        const int qb = li & 1;
-        if (lane == 0) {
-          if (li >= 2 && !W.wait(&B.q_empty[qb], ((li - 2) >> 1) & 1)) aborted = true;
-          if (!aborted) {
-            mbar_arrive_expect_tx(&B.q_full[qb], L::Q_BYTES);
-            uint8_t* dst = tiles + L::OFF_Q + qb * L::Q_BYTES;
-#pragma unroll
-            for (int h = 0; h < L::NH; ++h) tma_load_2d(dst + h * 8192, &p.tm_q, &B.q_full[qb], 64 * h, item * 64);
-            last_q = li;
-          }
-        }
-        aborted = __shfl_sync(0xffffffffu, aborted, 0);
-      }
       for (int t0 = 0; t0 < ntiles && !aborted; t0 += 16) {
         const int e = 2 * t0 + lane;
         int mine = (e < n) ? list[e] : 0;
@@ -265,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
           mine = 0;
         }
         const int tend = min(ntiles, t0 + 16);
-        for (int t = t0; t < tend; ++t, ++g) {
+        for (int t = t0; t < tend; ++t) {
           const int ca = __shfl_sync(0xffffffffu, mine, 2 * (t - t0));
           int cb = __shfl_sync(0xffffffffu, mine, 2 * (t - t0) + 1);
           if (2 * t + 1 >= n) cb = ca;  // odd tail: load a copy, the softmax masks it
@@ -284,274 +292,256 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
           }
           aborted = __shfl_sync(0xffffffffu, aborted, 0);
           if (aborted) break;
+          ++g;
         }
       }
     }
     if (bad && lane == 0) atomicOr(p.err, kErrBadIndex);
-    // Drain: wait for the copies this thread issued. Tiles 0..g-1 were
-    // issued (an aborted step breaks before issuing and before ++g); only the
-    // last use of each stage can still be in flight.
-    if (lane == 0) {
+    // Drain: steps 0..g-1 were issued; only the last use of each stage can be in flight.
+    if (lane == 0)
       for (int j = max(0, g - NS); j < g; ++j) W.drain_wait(&full[j % NS], (j / NS) & 1);
-      if (is_k && last_q >= 0)
-        for (int lj = max(0, last_q - 1); lj <= last_q; ++lj) W.drain_wait(&B.q_full[lj & 1], (lj >> 1) & 1);
-    }
   } else if (warp == 2) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, false, false);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(D, 64, true, true);
-      const uint32_t sQ = smem_u32(tiles + L::OFF_Q), sK = smem_u32(tiles + L::OFF_K),
-                     sV = smem_u32(tiles + L::OFF_V), sP = smem_u32(tiles + L::OFF_P);
+      constexpr uint32_t idesc_s = idesc_bf16_f32(64, 128, false, false);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(64, D, false, true);
+      const uint32_t sK = smem_u32(tiles + L::OFF_K), sV = smem_u32(tiles + L::OFF_V);
+      // K tile: K-major (rows = keys, 128 B per row segment); V tile: MN-major (rows = keys).
+      const uint64_t kdesc0 = sdesc_sw128(sK, 16, 1024);
+      const uint64_t vdesc0 = sdesc_sw128(sV, 16384, 1024);
       bool aborted = false, issued_any = false, bad = false;
       if (p.debug_stall && !W.wait(&B.stall, 0)) aborted = true;
-      int g = 0;
-      // O^T step for tile gg (first = first tile of its item).
-      auto issue_o = [&](int gg, bool first, int ob) -> bool {
-        const int vs = gg % kNV, pb = gg & 1;
-        if (!W.wait(&B.v_full[vs], (gg / kNV) & 1)) return false;
+      int g = 0;          // steps (S) issued
+      int li = 0;         // local item index
+      // The pending O step (issued after the next S).
+      bool have_prev = false, prev_first = false, prev_last = false;
+      int prev_g = 0, prev_li = 0;
+      auto issue_o = [&](int gg, bool first, bool last, int item_li) -> bool {
+        const int vs = gg % kVStages, pb = gg & 1;
+        if (!W.wait(&B.v_full[vs], (gg / kVStages) & 1)) return false;
         if (!W.wait(&B.p_full[pb], (gg >> 1) & 1)) return false;
+        if (first && item_li >= 1 && !W.wait(&B.o_empty, (item_li - 1) & 1)) return false;
         tc_fence_after();
+        const uint64_t vd = vdesc0 + (uint64_t)((vs * L::KV_BYTES) >> 4);
 #pragma unroll
-        for (int s = 0; s < 8; ++s) {  // 8 steps of 16 keys
-          const uint64_t ad = sdesc_sw128(sV + vs * L::KV_BYTES + s * 2048, 16384, 1024);
-          const uint64_t bd = sdesc_sw128(sP + pb * L::P_BYTES + s * 2048, 8192, 1024);
-          mma_bf16_ss(tO + ob * 64, ad, bd, idesc_o, (first && s == 0) ? 0u : 1u);
-        }
+        for (int s = 0; s < 8; ++s)  // 8 steps of 16 keys; P step s = 8 TMEM columns
+          mma_bf16_ts(tmem + kColO, tmem + kColS + 128u * pb + 8u * s, vd + (uint64_t)((s * 2048) >> 4), idesc_o,
+                      (first && s == 0) ? 0u : 1u);
         mma_commit(&B.v_empty[vs]);
-        mma_commit(&B.p_empty[pb]);
+        mma_commit(&B.o_step);
+        if (last) mma_commit(&B.o_full);
         return true;
       };
-      for (int li = 0, item = blockIdx.x; item < p.n_items && !aborted; ++li, item += gridDim.x) {
+      for (int item = blockIdx.x; item < p.n_items && !aborted; item += gridDim.x, ++li) {
         const int n = item_count(p, item, &bad);
         const int ntiles = (n + 1) >> 1;
-        const int qb = li & 1, ob = li & 1;
-        if (!W.wait(&B.q_full[qb], (li >> 1) & 1)) { aborted = true; break; }
-        if (li >= 2 && !W.wait(&B.o_empty[ob], ((li - 2) >> 1) & 1)) { aborted = true; break; }
+        const int qb = li & 1;
         for (int t = 0; t < ntiles; ++t, ++g) {
-          const int ks = g % kNK, sb = g & 1;
-          if (!W.wait(&B.k_full[ks], (g / kNK) & 1)) { aborted = true; break; }
-          if (g >= 2 && !W.wait(&B.s_empty[sb], ((g - 2) >> 1) & 1)) { aborted = true; break; }
+          if (t == 0 && !W.wait(&B.q_full[qb], (li >> 1) & 1)) { aborted = true; break; }
+          const int ks = g % kKStages, sb = g & 1;
+          if (!W.wait(&B.k_full[ks], (g / kKStages) & 1)) { aborted = true; break; }
           tc_fence_after();
+          const uint64_t kd = kdesc0 + (uint64_t)((ks * L::KV_BYTES) >> 4);
 #pragma unroll
-          for (int s = 0; s < D / 16; ++s) {  // steps of 16 along D
-            const uint32_t koff = (s >> 2) * 16384 + (s & 3) * 32;
-            const uint32_t qoff = (s >> 2) * 8192 + (s & 3) * 32;
-            const uint64_t ad = sdesc_sw128(sK + ks * L::KV_BYTES + koff, 16, 1024);
-            const uint64_t bd = sdesc_sw128(sQ + qb * L::Q_BYTES + qoff, 16, 1024);
-            mma_bf16_ss(tS + sb * 64, ad, bd, idesc_s, s > 0 ? 1u : 0u);
-          }
+          for (int s = 0; s < D / 16; ++s)  // steps of 16 along D; Q step s = 8 TMEM columns
+            mma_bf16_ts(tmem + kColS + 128u * sb, tmem + kColQ + kQCols * qb + 8u * s,
+                        kd + (uint64_t)(((s >> 2) * 16384 + (s & 3) * 32) >> 4), idesc_s, s > 0 ? 1u : 0u);
           issued_any = true;
           mma_commit(&B.k_empty[ks]);
           mma_commit(&B.s_full[sb]);
-          if (t > 0 && !issue_o(g - 1, t == 1, ob)) { aborted = true; break; }
+          if (have_prev && !issue_o(prev_g, prev_first, prev_last, prev_li)) { aborted = true; break; }
+          have_prev = true;
+          prev_g = g;
+          prev_first = (t == 0);
+          prev_last = (t == ntiles - 1);
+          prev_li = li;
         }
-        if (aborted) break;
-        if (!issue_o(g - 1, ntiles == 1, ob)) { aborted = true; break; }
-        mma_commit(&B.o_full[ob]);
       }
-      // Drain: all MMAs issued by this thread complete before TMEM is released.
+      if (!aborted && have_prev && !issue_o(prev_g, prev_first, prev_last, prev_li)) aborted = true;
+      // Drain: every MMA issued by this thread completes before TMEM is released.
       if (issued_any) {
         mma_commit(&B.drain);
         W.drain_wait(&B.drain, 0);
       }
     }
     __syncwarp();
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------ softmax + epilogue
-    const int sw = warp - 4;              // TMEM lane quarter
-    const int kr = sw * 32 + lane;        // key row of S^T / d row of O^T
-    const uint32_t lane_base = (uint32_t)(sw * 32) << 16;
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ softmax
+    const int quarter = warp & 3;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const float scale = p.scale_log2;
-    uint8_t* sP = tiles + L::OFF_P;
-    int g = 0;
     bool bad = false;
-    for (int li = 0, item = blockIdx.x; item < p.n_items; ++li, item += gridDim.x) {
-      const int bh = item / C, ci = item - bh * C;
+    int g = 0;
+    int li = 0;
+    for (int item = blockIdx.x; item < p.n_items; item += gridDim.x, ++li) {
       const int n = item_count(p, item, &bad);
       const int ntiles = (n + 1) >> 1;
-      const int ob = li & 1, qb = li & 1;
-      const int st = kr;  // softmax-group thread index 0..127
-      if (st < 64) {
-        sh.m_ref[st] = -INFINITY;
-        const int tok = cube_token(ci, st, p.H, p.W);
-        sh.tok[st] = tok;
-        sh.gc[st] = p.gate_c[(size_t)bh * p.N + tok];
-        sh.gf[st] = p.gate_f[(size_t)bh * p.N + tok];
-      }
-      float lp[64];
-#pragma unroll
-      for (int q = 0; q < 64; ++q) lp[q] = 0.f;
-      softmax_sync();
-
+      float m0 = -INFINITY, m1 = -INFINITY;  // reference max (scaled) of rows a and a+8
+      float l0 = 0.f, l1 = 0.f;              // this thread's share of the row sums
       for (int t = 0; t < ntiles; ++t, ++g) {
-        const int sb = g & 1, pb = g & 1;
+        const int sb = g & 1;
         W.wait(&B.s_full[sb], (g >> 1) & 1);
         tc_fence_after();
-        float x[64];
-        {
-          uint32_t r[32];
-          tmem_ld32(tS + sb * 64 + lane_base, r);
+        uint32_t r[64];
+        ld_16x256b_x16(tmem + kColS + 128u * sb + lane_base, r);
+        tmem_wait_ld();
+        const bool hi_valid = (2 * t + 1 < n);  // keys 64..127 (second cube) present
+        float x0 = -INFINITY, x1 = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          if (j < 8 || hi_valid) {
+            x0 = fmaxf(x0, fmaxf(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1])));
+            x1 = fmaxf(x1, fmaxf(__uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])));
+          }
+        }
+        x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, 1));
+        x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, 1));
+        x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, 2)) * scale;
+        x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, 2)) * scale;
+        // Lazy reference update per row.
+        float a0 = 1.f, a1 = 1.f;
+        const bool u0 = x0 > m0 + 8.0f, u1 = x1 > m1 + 8.0f;
+        if (u0) { a0 = fast_exp2(m0 - x0); m0 = x0; l0 *= a0; }
+        if (u1) { a1 = fast_exp2(m1 - x1); m1 = x1; l1 *= a1; }
+        if (t > 0 && __any_sync(0xffffffffu, u0 || u1)) {
+          // O holds steps < t of this item: wait for the previous O step, rescale rows.
+          W.wait(&B.o_step, (g - 1) & 1);
+          tc_fence_after();
+          uint32_t o[64];
+          if (D == 128) ld_16x256b_x16(tmem + kColO + lane_base, o);
+          else ld_16x256b_x8(tmem + kColO + lane_base, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int q = 0; q < 32; ++q) x[q] = __uint_as_float(r[q]) * scale;
-          tmem_ld32(tS + sb * 64 + 32 + lane_base, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int q = 0; q < 32; ++q) x[32 + q] = __uint_as_float(r[q]) * scale;
+          for (int j = 0; j < D / 8; ++j) {
+            o[4 * j] = __float_as_uint(__uint_as_float(o[4 * j]) * a0);
+            o[4 * j + 1] = __float_as_uint(__uint_as_float(o[4 * j + 1]) * a0);
+            o[4 * j + 2] = __float_as_uint(__uint_as_float(o[4 * j + 2]) * a1);
+            o[4 * j + 3] = __float_as_uint(__uint_as_float(o[4 * j + 3]) * a1);
+          }
+          if (D == 128) st_16x256b_x16(tmem + kColO + lane_base, o);
+          else st_16x256b_x8(tmem + kColO + lane_base, o);
+          tmem_wait_st();
         }
+        // P = 2^(s*scale - m), packed to bf16 pairs (keys c, c+1 -> P column c/2).
+        uint32_t pk[32];
+        const float nm0 = -m0, nm1 = -m1;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const bool v = (j < 8) || hi_valid;
+          const float p00 = v ? fast_exp2(fmaf(__uint_as_float(r[4 * j]), scale, nm0)) : 0.f;
+          const float p01 = v ? fast_exp2(fmaf(__uint_as_float(r[4 * j + 1]), scale, nm0)) : 0.f;
+          const float p10 = v ? fast_exp2(fmaf(__uint_as_float(r[4 * j + 2]), scale, nm1)) : 0.f;
+          const float p11 = v ? fast_exp2(fmaf(__uint_as_float(r[4 * j + 3]), scale, nm1)) : 0.f;
+          l0 += p00 + p01;
+          l1 += p10 + p11;
+          __nv_bfloat162 h0 = __floats2bfloat162_rn(p00, p01);
+          __nv_bfloat162 h1 = __floats2bfloat162_rn(p10, p11);
+          pk[2 * j] = *reinterpret_cast<uint32_t*>(&h0);
+          pk[2 * j + 1] = *reinterpret_cast<uint32_t*>(&h1);
+        }
+        st_16x128b_x16(tmem + kColS + 128u * sb + lane_base, pk);
+        tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&B.s_empty[sb]);
-        const bool valid = (kr < 64) || (2 * t + 1 < n);
-        // Does any score exceed the current reference max by more than 2^8?
-        bool need = false;
-#pragma unroll
-        for (int q4 = 0; q4 < 16; ++q4) {
-          const float4 m4 = *reinterpret_cast<const float4*>(&sh.m_ref[4 * q4]);
-          need |= (x[4 * q4 + 0] - m4.x > 8.0f) | (x[4 * q4 + 1] - m4.y > 8.0f) |
-                  (x[4 * q4 + 2] - m4.z > 8.0f) | (x[4 * q4 + 3] - m4.w > 8.0f);
-        }
-        need = softmax_sync_or(valid && need);
-        if (need) {
-          // Exact column max over the 128 keys of this step -> new reference.
-          float cm[64];
-#pragma unroll
-          for (int q = 0; q < 64; ++q) cm[q] = valid ? x[q] : -INFINITY;
-          warp_colreduce64<true>(cm, lane);
-          sh.red[sw][2 * lane] = cm[0];
-          sh.red[sw][2 * lane + 1] = cm[1];
-          softmax_sync();
-          if (st < 64) {
-            const float c = fmaxf(fmaxf(sh.red[0][st], sh.red[1][st]), fmaxf(sh.red[2][st], sh.red[3][st]));
-            const float mo = sh.m_ref[st];
-            const float mn = fmaxf(mo, c);
-            sh.alpha[st] = fast_exp2(mo - mn);  // 0 when mo = -inf
-            sh.m_ref[st] = mn;
-          }
-          softmax_sync();
-#pragma unroll
-          for (int q = 0; q < 64; ++q) lp[q] *= sh.alpha[q];
-          if (t > 0) {
-            // O^T holds steps < t of this item: rescale its query columns once
-            // the previous step's MMA has completed. All lanes take part in
-            // the (warp-collective) TMEM load/store.
-            W.wait(&B.p_empty[(g - 1) & 1], ((g - 1) >> 1) & 1);
-            tc_fence_after();
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-              uint32_t r[32];
-              const uint32_t a = tO + ob * 64 + half * 32 + lane_base;
-              tmem_ld32(a, r);
-              tmem_wait_ld();
-#pragma unroll
-              for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(__uint_as_float(r[q]) * sh.alpha[half * 32 + q]);
-              tmem_st32(a, r);
-            }
-            tmem_wait_st();
-          }
-        }
-        // p = 2^(x - m_ref), accumulated into the row-sum partials; x is reused for p.
-#pragma unroll
-        for (int q4 = 0; q4 < 16; ++q4) {
-          const float4 m4 = *reinterpret_cast<const float4*>(&sh.m_ref[4 * q4]);
-          const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int q = 4 * q4 + e;
-            const float pq = valid ? fast_exp2(x[q] - mm[e]) : 0.f;
-            lp[q] += pq;
-            x[q] = pq;
-          }
-        }
-        // P^T row kr -> shared memory (MN-major, 128-byte swizzle), once the
-        // MMA that read this buffer two steps ago has completed.
-        if (g >= 2) W.wait(&B.p_empty[pb], ((g - 2) >> 1) & 1);
-        uint8_t* prow = sP + pb * L::P_BYTES + kr * 128;
-#pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
-          uint32_t w4[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            __nv_bfloat162 h = __floats2bfloat162_rn(x[8 * c8 + 2 * e], x[8 * c8 + 2 * e + 1]);
-            w4[e] = *reinterpret_cast<uint32_t*>(&h);
-          }
-          *reinterpret_cast<uint4*>(prow + ((c8 ^ (kr & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&B.p_full[pb]);
+        if (lane == 0) mbar_arrive(&B.p_full[sb]);
       }
-
-      // ---------------------------------------------------------- epilogue
-      warp_colreduce64<false>(lp, lane);
-      sh.red[sw][2 * lane] = lp[0];
-      sh.red[sw][2 * lane + 1] = lp[1];
-      softmax_sync();
-      if (st < 64) sh.inv_l[st] = 1.0f / (sh.red[0][st] + sh.red[1][st] + sh.red[2][st] + sh.red[3][st]);
-      softmax_sync();
-      W.wait(&B.o_full[ob], (li >> 1) & 1);
-      tc_fence_after();
-      const bool has_d = (D == 128) || (lane < 16);
-      const int d = (D == 128) ? kr : sw * 16 + lane;
-      float o[64];
-      {
-        uint32_t r[32];
-        tmem_ld32(tO + ob * 64 + lane_base, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int q = 0; q < 32; ++q) o[q] = __uint_as_float(r[q]);
-        tmem_ld32(tO + ob * 64 + 32 + lane_base, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int q = 0; q < 32; ++q) o[32 + q] = __uint_as_float(r[q]);
+      // Row sums of the item -> 1/l for the epilogue.
+      l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+      l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+      if ((lane & 3) == 0) {
+        const int row = quarter * 16 + (lane >> 2);
+        sh.inv_l[li & 1][row] = 1.0f / l0;
+        sh.inv_l[li & 1][row + 8] = 1.0f / l1;
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&B.l_full[li & 1]);
+    }
+    if (bad && tid == 128) atomicOr(p.err, kErrBadIndex);
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ epilogue (+ Q loads)
+    const int quarter = warp & 3;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const int ra = quarter * 16 + (lane >> 2);  // rows ra and ra + 8 of the item
+    const int tq = lane & 3;
+    const int est = tid - 256;                  // 0..127 within the epilogue group
+    uint8_t* stage = tiles + L::OFF_STAGE;
+    // Q of an item -> TMEM buffer b (A operand layout: row per lane, bf16 pairs per column).
+    auto load_q = [&](int item, int b) {
+      const __nv_bfloat16* qsrc = p.q_cube + (size_t)item * 64 * D;
+      uint32_t r[64];
+#pragma unroll
+      for (int j = 0; j < D / 16; ++j) {
+        const uint2 va = *reinterpret_cast<const uint2*>(qsrc + (size_t)ra * D + 16 * j + 4 * tq);
+        const uint2 vb = *reinterpret_cast<const uint2*>(qsrc + (size_t)(ra + 8) * D + 16 * j + 4 * tq);
+        r[4 * j] = va.x; r[4 * j + 1] = va.y; r[4 * j + 2] = vb.x; r[4 * j + 3] = vb.y;
+      }
+      const uint32_t ta = tmem + kColQ + (uint32_t)(D / 2) * b + lane_base;
+      if (D == 128) st_16x256b_x8(ta, r);
+      else st_16x256b_x4(ta, reinterpret_cast<uint32_t(&)[32]>(r));
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&B.o_empty[ob]);
-      const float ocd = has_d ? p.oc[((size_t)bh * C + ci) * D + d] : 0.f;
+      if (lane == 0) mbar_arrive(&B.q_full[b]);
+    };
+    if (blockIdx.x < p.n_items) load_q(blockIdx.x, 0);
+    if (blockIdx.x + gridDim.x < p.n_items) load_q(blockIdx.x + gridDim.x, 1);
+    int li = 0;
+    for (int item = blockIdx.x; item < p.n_items; item += gridDim.x, ++li) {
+      const int bh = item / C, ci = item - bh * C;
+      // per-item constants: gates of rows ra, ra+8 and this thread's coarse-output columns
+      const int tok0 = cube_token(ci, ra, p.H, p.W), tok1 = cube_token(ci, ra + 8, p.H, p.W);
+      const float gc0 = p.gate_c[(size_t)bh * p.N + tok0], gf0 = p.gate_f[(size_t)bh * p.N + tok0];
+      const float gc1 = p.gate_c[(size_t)bh * p.N + tok1], gf1 = p.gate_f[(size_t)bh * p.N + tok1];
+      const float* ocrow = p.oc + ((size_t)bh * C + ci) * D;
+      W.wait(&B.l_full[li & 1], (li >> 1) & 1);
+      const float il0 = sh.inv_l[li & 1][ra], il1 = sh.inv_l[li & 1][ra + 8];
+      W.wait(&B.o_full, li & 1);
+      tc_fence_after();
+      uint32_t o[64];
+      if (D == 128) ld_16x256b_x16(tmem + kColO + lane_base, o);
+      else ld_16x256b_x8(tmem + kColO + lane_base, o);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&B.o_empty);
+      // All S steps of this item are complete, so its Q buffer takes the item after next.
+      if (item + 2 * gridDim.x < p.n_items) load_q(item + 2 * gridDim.x, li & 1);
+      if (p.out_fine) {
 #pragma unroll
-      for (int q = 0; q < 64; ++q) o[q] *= sh.inv_l[q];
-      if (p.out_fine && has_d) {
-        for (int q = 0; q < 64; ++q) p.out_fine[((size_t)bh * p.N + sh.tok[q]) * D + d] = o[q];
-      }
-      uint8_t* stage = tiles + L::OFF_Q + qb * L::Q_BYTES;  // Q buffer of this item, free now
-      if (p.out) {
-        // Gated combine, then pair lanes (d, d+1) so each lane writes 4 bytes.
-        const bool odd = lane & 1;
-#pragma unroll
-        for (int q2 = 0; q2 < 32; ++q2) {
-          const int qa = 2 * q2, qb2 = 2 * q2 + 1;
-          const float va = sh.gc[qa] * ocd + sh.gf[qa] * o[qa];
-          const float vb = sh.gc[qb2] * ocd + sh.gf[qb2] * o[qb2];
-          const float send = odd ? va : vb;
-          const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
-          if (has_d) {
-            // even lane: (q=qa: d, d+1); odd lane: (q=qb2: d-1, d)
-            const int q = odd ? qb2 : qa;
-            const int d0 = odd ? d - 1 : d;
-            const __nv_bfloat162 h = odd ? __floats2bfloat162_rn(recv, vb) : __floats2bfloat162_rn(va, recv);
-            *reinterpret_cast<__nv_bfloat162*>(stage + (q * D + d0) * 2) = h;
-          }
+        for (int j = 0; j < D / 8; ++j) {
+          const int d = 8 * j + 2 * tq;
+          *reinterpret_cast<float2*>(p.out_fine + ((size_t)bh * p.N + tok0) * D + d) =
+              make_float2(__uint_as_float(o[4 * j]) * il0, __uint_as_float(o[4 * j + 1]) * il0);
+          *reinterpret_cast<float2*>(p.out_fine + ((size_t)bh * p.N + tok1) * D + d) =
+              make_float2(__uint_as_float(o[4 * j + 2]) * il1, __uint_as_float(o[4 * j + 3]) * il1);
         }
       }
-      softmax_sync();
       if (p.out) {
+#pragma unroll
+        for (int j = 0; j < D / 8; ++j) {
+          const int d = 8 * j + 2 * tq;
+          const float2 oc = *reinterpret_cast<const float2*>(ocrow + d);
+          const __nv_bfloat162 h0 = __floats2bfloat162_rn(gc0 * oc.x + gf0 * __uint_as_float(o[4 * j]) * il0,
+                                                          gc0 * oc.y + gf0 * __uint_as_float(o[4 * j + 1]) * il0);
+          const __nv_bfloat162 h1 = __floats2bfloat162_rn(gc1 * oc.x + gf1 * __uint_as_float(o[4 * j + 2]) * il1,
+                                                          gc1 * oc.y + gf1 * __uint_as_float(o[4 * j + 3]) * il1);
+          *reinterpret_cast<__nv_bfloat162*>(stage + (ra * D + d) * 2) = h0;
+          *reinterpret_cast<__nv_bfloat162*>(stage + ((ra + 8) * D + d) * 2) = h1;
+        }
+        epi_sync();
         constexpr int CPR = D / 8;  // 16-byte chunks per row
 #pragma unroll
         for (int u = 0; u < (64 * CPR) / 128; ++u) {
-          const int c = st + 128 * u;
-          const int q = c / CPR, off = c % CPR;
+          const int cidx = est + 128 * u;
+          const int q = cidx / CPR, off = cidx % CPR;
           const uint4 v = *reinterpret_cast<const uint4*>(stage + (q * D + off * 8) * 2);
-          *reinterpret_cast<uint4*>(p.out + ((size_t)bh * p.N + sh.tok[q]) * D + off * 8) = v;
+          *reinterpret_cast<uint4*>(p.out + ((size_t)bh * p.N + cube_token(ci, q, p.H, p.W)) * D + off * 8) = v;
         }
+        epi_sync();
       }
-      fence_proxy_async_smem();
-      softmax_sync();
-      if (lane == 0) mbar_arrive(&B.q_empty[qb]);
     }
-    (void)bad;
   }
 
   tc_fence_before();
