@@ -17,7 +17,7 @@ struct vsa_plan_s {
   int BH, N, C, kcap;
   char* ws;
   vsa_workspace_layout_t lay;
-  CUtensorMap tm_k, tm_v;
+  CUtensorMap tm_q, tm_k, tm_v;
   int num_sms;
   cudaStream_t last_stream;
   uint64_t wait_ns;
@@ -151,10 +151,10 @@ vsa_status run_common(vsa_plan_t P, const void* q, const void* k, const void* v,
   if (vsa::launch_coarse(cp, st) != cudaSuccess) return VSA_ERR_CUDA;
 
   vsa::FineParams fp{};
-  fp.tm_k = P->tm_k; fp.tm_v = P->tm_v;
-  fp.q_cube = gp.dst[0];
+  fp.tm_q = P->tm_q; fp.tm_k = P->tm_k; fp.tm_v = P->tm_v;
   fp.idx = select ? idx_out : idx_in;
-  fp.cnt = select ? cp.cnt : cnt_in;
+  // Top-K rows all hold exactly topk ids: the fine kernel then needs no counts.
+  fp.cnt = select ? (P->cfg.topk > 0 ? nullptr : cp.cnt) : cnt_in;
   fp.oc = cp.oc;
   fp.gate_c = gate_c; fp.gate_f = gate_f;
   fp.out = static_cast<__nv_bfloat16*>(out);
@@ -229,7 +229,8 @@ vsa_status vsa_plan(vsa_plan_t* out, const vsa_config* cfg, void* workspace, siz
   P->wait_ns = 1000000000ull;
   P->debug_stall = 0;
   const size_t rows = (size_t)P->BH * P->N;
-  vsa_status e = encode_map(&P->tm_k, P->ws + L.k_cube, rows, cfg->D);
+  vsa_status e = encode_map(&P->tm_q, P->ws + L.q_cube, rows, cfg->D);
+  if (e == VSA_OK) e = encode_map(&P->tm_k, P->ws + L.k_cube, rows, cfg->D);
   if (e == VSA_OK) e = encode_map(&P->tm_v, P->ws + L.v_cube, rows, cfg->D);
   if (e == VSA_OK && cudaMemset(P->ws + L.err, 0, 16) != cudaSuccess) e = VSA_ERR_CUDA;
   if (e != VSA_OK) {
@@ -370,7 +371,8 @@ vsa_status vsa_forward_noalloc(const void* q, const void* k, const void* v, cons
   P.num_sms = sms;
   P.wait_ns = 1000000000ull;
   const size_t rows = (size_t)P.BH * P.N;
-  s = encode_map(&P.tm_k, P.ws + L.k_cube, rows, D);
+  s = encode_map(&P.tm_q, P.ws + L.q_cube, rows, D);
+  if (s == VSA_OK) s = encode_map(&P.tm_k, P.ws + L.k_cube, rows, D);
   if (s == VSA_OK) s = encode_map(&P.tm_v, P.ws + L.v_cube, rows, D);
   if (s != VSA_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

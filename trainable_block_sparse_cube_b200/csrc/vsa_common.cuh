@@ -46,8 +46,7 @@ struct CoarseParams {
 };
 
 struct FineParams {
-  CUtensorMap tm_k, tm_v;        // 2-D maps over the cube-major K and V copies, rows of D bf16
-  const __nv_bfloat16* q_cube;   // cube-major Q copy [BH, C, 64, D]
+  CUtensorMap tm_q, tm_k, tm_v;  // 2-D maps over the cube-major copies, rows of D bf16
   const int32_t* idx;            // [BH, C, kcap]
   const int32_t* cnt;            // [BH, C] or null (then every row has kcap ids)
   const float* oc;               // [BH, C, D]
