@@ -234,6 +234,7 @@ struct alignas(16) Shared {
   Bars bar;
   uint32_t tmem_base;
   int abort_flag;
+  int issue_lock;                     // held by an MMA issuer while it enqueues a block
   int epi_pick;                       // stream whose item the epilogue handles next
   alignas(16) float inv_l[2][2][64];  // [stream][item parity][row]
 };
@@ -251,6 +252,22 @@ struct Waiter {
 #pragma unroll 1
       for (int i = 0; i < 64; ++i)
         if (mbar_try_wait(bar, parity)) return true;
+      if (*(volatile int*)&sh->abort_flag) return false;
+      if (globaltimer_ns() - t0 > limit) {
+        *(volatile int*)&sh->abort_flag = 1;
+        atomicOr(err, kErrTimeout);
+        return false;
+      }
+    }
+  }
+  // Bounded acquisition of a shared-memory spin lock; false on timeout or abort.
+  __device__ __forceinline__ bool acquire(int* lock) const {
+    if (atomicCAS(lock, 0, 1) == 0) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+#pragma unroll 1
+      for (int i = 0; i < 64; ++i)
+        if (atomicCAS(lock, 0, 1) == 0) return true;
       if (*(volatile int*)&sh->abort_flag) return false;
       if (globaltimer_ns() - t0 > limit) {
         *(volatile int*)&sh->abort_flag = 1;
@@ -341,6 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
     }
     mbar_init(&B.stall, 1);
     sh.abort_flag = 0;
+    sh.issue_lock = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -440,10 +458,14 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
       Cursor c;
       cursor_init(p, c, s);
       int j = 0;  // steps of this stream
-      // S of the step at the cursor: Q buffer of the item, K of the step.
-      bool s_ok = !aborted && c.live;
-      if (s_ok) s_ok = W.wait(&B.q_full[s][0], 0) && W.wait(&B.k_full[s], 0);
-      if (s_ok) {
+      // Each block ([S(0)], then [O(j), S(j+1)]) is enqueued under the issue
+      // lock once all its operands are ready, so the two streams' blocks reach
+      // the tensor core whole and in turn: one stream's S completes a block
+      // ahead of the other's and the two softmax groups run staggered instead
+      // of contending for the same units.
+      bool ok = !aborted && c.live;
+      if (ok) ok = W.wait(&B.q_full[s][0], 0) && W.wait(&B.k_full[s], 0) && W.acquire(&sh.issue_lock);
+      if (ok) {
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
@@ -451,16 +473,22 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
                       kdesc + (uint64_t)(((k >> 2) * 16384 + (k & 3) * 32) >> 4), idesc_s, k > 0 ? 1u : 0u);
         mma_commit(&B.k_empty[s]);
         mma_commit(&B.s_full[s]);
+        atomicExch(&sh.issue_lock, 0);
         issued_any = true;
       } else if (c.live) {
         aborted = true;
       }
       while (!aborted && c.live) {
-        // O of step j (P in TMEM, V in smem).
+        // O of step j (P in TMEM, V in smem), then S of step j + 1.
         const bool first = (c.t == 0), last = (c.t == c.ntiles - 1);
         const int is = c.is;
+        Cursor nx = c;
+        cursor_next(p, nx);
+        const int qb = nx.is & 1;
         if (!W.wait(&B.v_full[s], j & 1) || !W.wait(&B.p_full[s], j & 1) ||
-            (first && is >= 1 && !W.wait(&B.o_empty[s], (is - 1) & 1))) {
+            (first && is >= 1 && !W.wait(&B.o_empty[s], (is - 1) & 1)) ||
+            (nx.live && nx.t == 0 && !W.wait(&B.q_full[s][qb], (nx.is >> 1) & 1)) ||
+            (nx.live && !W.wait(&B.k_full[s], (j + 1) & 1)) || !W.acquire(&sh.issue_lock)) {
           aborted = true;
           break;
         }
@@ -470,23 +498,18 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
           mma_bf16_ts(tO, tS + 8u * k, vdesc + (uint64_t)((k * 2048) >> 4), idesc_o, (first && k == 0) ? 0u : 1u);
         mma_commit(&B.v_empty[s]);
         if (last) mma_commit(&B.o_full[s]);
-        ++j;
-        cursor_next(p, c);
-        if (!c.live) break;
-        // S of step j.
-        const int qb = c.is & 1;
-        if ((c.t == 0 && !W.wait(&B.q_full[s][qb], (c.is >> 1) & 1)) || !W.wait(&B.k_full[s], j & 1)) {
-          aborted = true;
-          break;
-        }
-        tc_fence_after();
-        const uint64_t qd = qdesc0 + (uint64_t)((qb * L::Q_BYTES) >> 4);
+        if (nx.live) {
+          const uint64_t qd = qdesc0 + (uint64_t)((qb * L::Q_BYTES) >> 4);
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k)  // steps of 16 along D
-          mma_bf16_ss(tS, qd + (uint64_t)(((k >> 2) * 8192 + (k & 3) * 32) >> 4),
-                      kdesc + (uint64_t)(((k >> 2) * 16384 + (k & 3) * 32) >> 4), idesc_s, k > 0 ? 1u : 0u);
-        mma_commit(&B.k_empty[s]);
-        mma_commit(&B.s_full[s]);
+          for (int k = 0; k < D / 16; ++k)  // steps of 16 along D
+            mma_bf16_ss(tS, qd + (uint64_t)(((k >> 2) * 8192 + (k & 3) * 32) >> 4),
+                        kdesc + (uint64_t)(((k >> 2) * 16384 + (k & 3) * 32) >> 4), idesc_s, k > 0 ? 1u : 0u);
+          mma_commit(&B.k_empty[s]);
+          mma_commit(&B.s_full[s]);
+        }
+        atomicExch(&sh.issue_lock, 0);
+        ++j;
+        c = nx;
       }
       // Drain: every MMA issued by this thread completes before TMEM is released.
       if (issued_any) {
