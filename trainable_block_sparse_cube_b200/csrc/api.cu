@@ -18,6 +18,8 @@ struct vsa_plan_s {
   char* ws;
   vsa_workspace_layout_t lay;
   CUtensorMap tm_q, tm_k, tm_v;
+  CUtensorMap tm_out;       // output map, encoded for the output pointer tm_out_for
+  const void* tm_out_for;
   int num_sms;
   cudaStream_t last_stream;
   uint64_t wait_ns;
@@ -107,6 +109,22 @@ vsa_status encode_map(CUtensorMap* m, void* base, size_t rows, int D) {
   return r == CUDA_SUCCESS ? VSA_OK : VSA_ERR_CUDA;
 }
 
+// 5-D map over the raster output [BH][T][H][W][D] bf16: a box is one cube's
+// 4 x 4 x 4 tokens by 64 channels, stored from a 128-byte-swizzled tile.
+vsa_status encode_out_map(CUtensorMap* m, void* base, const vsa_config& c, int BH) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return VSA_ERR_CUDA;
+  const cuuint64_t D = (cuuint64_t)c.D;
+  cuuint64_t dims[5] = {D, (cuuint64_t)c.W, (cuuint64_t)c.H, (cuuint64_t)c.T, (cuuint64_t)BH};
+  cuuint64_t strides[4] = {D * 2, (cuuint64_t)c.W * D * 2, (cuuint64_t)c.H * c.W * D * 2,
+                           (cuuint64_t)c.T * c.H * c.W * D * 2};
+  cuuint32_t box[5] = {64, 4, 4, 4, 1};
+  cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? VSA_OK : VSA_ERR_CUDA;
+}
+
 vsa_status run_common(vsa_plan_t P, const void* q, const void* k, const void* v, const float* gate_c,
                       const float* gate_f, bool select, const int32_t* idx_in, const int32_t* cnt_in, int32_t* idx_out,
                       int32_t* cnt_out, void* out, float* out_coarse, float* out_fine, void* stream) {
@@ -152,6 +170,14 @@ vsa_status run_common(vsa_plan_t P, const void* q, const void* k, const void* v,
 
   vsa::FineParams fp{};
   fp.tm_q = P->tm_q; fp.tm_k = P->tm_k; fp.tm_v = P->tm_v;
+  if (out) {
+    if (P->tm_out_for != out) {
+      const vsa_status e = encode_out_map(&P->tm_out, out, c, P->BH);
+      if (e != VSA_OK) return e;
+      P->tm_out_for = out;
+    }
+    fp.tm_out = P->tm_out;
+  }
   fp.idx = select ? idx_out : idx_in;
   // Top-K rows all hold exactly topk ids: the fine kernel then needs no counts.
   fp.cnt = select ? (P->cfg.topk > 0 ? nullptr : cp.cnt) : cnt_in;

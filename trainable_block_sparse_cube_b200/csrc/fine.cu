@@ -14,18 +14,13 @@
 //   S[64 q x 128 keys] = Q . K_pair^T     tcgen05.mma M=64, N=128 (Q, K in smem)
 //   O[64 q x D]       += P . V_pair       tcgen05.mma M=64, N=D   (P in TMEM, V in smem)
 //
-// Two item streams run interleaved (the CTA's even and odd items), each with
-// its own TMA producer warp, K and V buffers, MMA-issuing warp, softmax
-// warpgroup, S/P buffer and O accumulator in tensor memory, so the tensor core
-// always has the other stream's work while one stream's softmax runs. The
-// streams share nothing but the tensor core and the epilogue: each issuer
-// keeps its own stream's order [S(0)], [O(j), S(j+1)], ... . A tcgen05.mma
-// issue occupies the issuing thread for about as long as an M=64 N=128 MMA
-// runs, so a single issuing thread leaves no slack for its waits; one issuing
-// thread per stream keeps the tensor core fed while the other one waits.
-// Because a tcgen05 commit covers every earlier MMA of the issuing thread,
-// "S(j+1) complete" also means "O(j) complete": when a softmax warp sees its
-// next S it may overwrite P in place and rescale O.
+// Tensor memory holds two S/P buffers and two O accumulators, so S of step
+// j+1 runs on the tensor core while the softmax works on step j, and the
+// epilogue reads an item's O while the next item accumulates into the other
+// buffer. All eight softmax warps work on the same step: warp w handles the
+// rows of TMEM lane quarter w % 4 and the key half w / 4 (64 keys). The two
+// warps that share rows agree on the row statistics through a 64-thread
+// named barrier.
 //
 // The M=64 accumulators occupy 16 lanes of each 32-lane TMEM quarter; the
 // 16-lane tcgen05.ld/st shapes spread those lanes over a whole warp: with
@@ -36,13 +31,16 @@
 // the reference max of a row moves only when a score exceeds it by more than
 // 2^8, after the first step of an item rarely.
 //
+// A tcgen05.mma issue occupies the issuing thread for about as long as an
+// M=64 N=128 MMA runs, so the S and the O MMAs come from two issuing threads.
+//
 // Warp roles (512 threads):
-//   warps 0, 1  TMA producer of stream 0, 1: K and V of a step (one buffer
-//               each; two issuing threads keep the L2 -> SM stream full)
-//   warps 2, 3  single-thread tcgen05.mma issuer of stream 0, 1 (warp 2 also
-//               allocates tensor memory)
-//   warps 4-7   softmax of stream 0     warps 8-11  softmax of stream 1
-//   warps 12-15 epilogue: Q loads, 1/l and gates, output rows
+//   warp 0      TMA producer of K (3-stage ring of steps)
+//   warp 1      TMA producer of V (2-stage ring of steps)
+//   warp 2      issuer of the S MMAs (also allocates tensor memory)
+//   warp 3      issuer of the O MMAs
+//   warps 4-11  softmax
+//   warps 12-15 epilogue: Q loads, gates and coarse rows, output tiles (TMA)
 //
 // Every mbarrier wait is bounded (plan wait limit). A wait that gives up
 // records kErrTimeout, sets a CTA-wide abort flag that makes every later wait
@@ -58,8 +56,10 @@ namespace {
 using namespace ptx;
 
 constexpr int kThreads = 512;
+constexpr int kKStages = 3;  // K ring depth (steps of two cubes)
+constexpr int kVStages = 2;  // V ring depth
 constexpr uint32_t kTmemCols = 512;
-// TMEM columns: S/P of stream s at 128 s, O of stream s at 256 + 128 s.
+// TMEM columns: S/P buffer b at 128 b, O buffer b at 256 + 128 b.
 constexpr uint32_t kColSP = 0, kColO = 256;
 
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -69,6 +69,20 @@ __device__ __forceinline__ float fast_exp2(float x) {
 }
 
 __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 3, 128;" ::: "memory"); }
+// The two softmax warps of lane quarter q (warps 4+q and 8+q) use barrier 4+q.
+__device__ __forceinline__ void pair_sync(int q) { asm volatile("bar.sync %0, 64;" ::"r"(4 + q) : "memory"); }
+__device__ __forceinline__ bool pair_any(int q, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, o;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred o, %2, 64, p;\n\t"
+      "selp.u32 %0, 1, 0, o;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(4 + q)
+      : "memory");
+  return r != 0;
+}
 
 // Register split between warpgroups (the launch gives every thread 128):
 // warps 0-3 (producers, MMA issuers) 72, softmax 152, epilogue 136;
@@ -82,19 +96,7 @@ __device__ __forceinline__ void regs_inc() { asm volatile("setmaxnreg.inc.sync.a
 // ---- 16-lane TMEM shapes (lanes base..base+15 of the warp's quarter) ----
 #define VSA_O4(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3])
 #define VSA_I4(i) "r"(r[i]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3])
-// .16x256b.x16: 128 columns; r[4j..4j+3] = (row a: col c, c+1; row a+8: col c, c+1), c = 8j + 2(t%4).
-__device__ __forceinline__ void ld_16x256b_x16(uint32_t taddr, uint32_t (&r)[64]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.16x256b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
-      "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
-      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
-      : VSA_O4(0), VSA_O4(4), VSA_O4(8), VSA_O4(12), VSA_O4(16), VSA_O4(20), VSA_O4(24), VSA_O4(28),
-        VSA_O4(32), VSA_O4(36), VSA_O4(40), VSA_O4(44), VSA_O4(48), VSA_O4(52), VSA_O4(56), VSA_O4(60)
-      : "r"(taddr));
-}
-// .16x256b.x8: 64 columns, 32 registers.
+// .16x256b.x8: 64 columns; r[4j..4j+3] = (row a: col c, c+1; row a+8: col c, c+1), c = 8j + 2(t%4).
 __device__ __forceinline__ void ld_16x256b_x8(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.16x256b.x8.b32 "
@@ -111,13 +113,12 @@ __device__ __forceinline__ void st_16x256b_x8(uint32_t taddr, const uint32_t (&r
       VSA_I4(0), VSA_I4(4), VSA_I4(8), VSA_I4(12), VSA_I4(16), VSA_I4(20), VSA_I4(24), VSA_I4(28)
       : "memory");
 }
-// .16x128b.x16: 64 columns; r[2j] -> (row a, col 4j + t%4), r[2j+1] -> (row a+8, same col).
-__device__ __forceinline__ void st_16x128b_x16(uint32_t taddr, const uint32_t (&r)[32]) {
+// .16x128b.x8: 32 columns; r[2j] -> (row a, col 4j + t%4), r[2j+1] -> (row a+8, same col).
+__device__ __forceinline__ void st_16x128b_x8(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
-      "tcgen05.st.sync.aligned.16x128b.x16.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      VSA_I4(0), VSA_I4(4), VSA_I4(8), VSA_I4(12), VSA_I4(16), VSA_I4(20), VSA_I4(24), VSA_I4(28)
+      "tcgen05.st.sync.aligned.16x128b.x8.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      VSA_I4(0), VSA_I4(4), VSA_I4(8), VSA_I4(12)
       : "memory");
 }
 #undef VSA_O4
@@ -128,7 +129,7 @@ __device__ __forceinline__ void st_16x128b_x16(uint32_t taddr, const uint32_t (&
 // bits) and f in [-1/2, 1/2]; 2^f is a cubic fitted by weighted least squares
 // (relative error) on Chebyshev nodes of [-1/2, 1/2], max relative error
 // 7.8e-5, far below the bf16 rounding of P; 2^n is added to the exponent
-// field. Offloads part of the exponentials from the 16-per-clock MUFU units.
+// field. Offloads part of the exponentials from the MUFU units.
 __device__ __forceinline__ float poly_exp2(float x) {
   x = fminf(fmaxf(x, -126.f), 64.f);
   const float t = __fadd_rn(x, 12582912.f);
@@ -139,19 +140,19 @@ __device__ __forceinline__ float poly_exp2(float x) {
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
-// Softmax numerators of one 128-key step for the thread's rows a and a+8
-// (register layout of ld_16x256b_x16): P = 2^(s*scale - m), packed to bf16
+// Softmax numerators of one 64-key half step for the thread's rows a and a+8
+// (register layout of ld_16x256b_x8): P = 2^(s*scale - m), packed to bf16
 // pairs (keys c, c+1 -> P column c/2), and the thread's partial row sums.
 // With POLY one column group in four takes the FMA-pipe exponential; masked
 // (-inf) scores need the exact zero of the MUFU path.
 template <bool POLY>
-__device__ __forceinline__ void exp_pack(const uint32_t (&r)[64], float scale, float m0, float m1,
-                                         uint32_t (&pk)[32], float& s0, float& s1) {
+__device__ __forceinline__ void exp_pack(const uint32_t (&r)[32], float scale, float m0, float m1,
+                                         uint32_t (&pk)[16], float& s0, float& s1) {
   const float nm0 = -m0, nm1 = -m1;
   s0 = 0.f;
   s1 = 0.f;
 #pragma unroll
-  for (int j = 0; j < 16; ++j) {
+  for (int j = 0; j < 8; ++j) {
     const bool poly = POLY && (j & 3) == 3;
     const float x00 = fmaf(__uint_as_float(r[4 * j]), scale, nm0);
     const float x01 = fmaf(__uint_as_float(r[4 * j + 1]), scale, nm0);
@@ -170,24 +171,19 @@ __device__ __forceinline__ void exp_pack(const uint32_t (&r)[64], float scale, f
   }
 }
 
-// Unscaled maxima of rows a and a+8 over the whole 128-key step (the four
-// threads of a row combine through shuffles).
-__device__ __forceinline__ void row_max(const uint32_t (&r)[64], float& x0, float& x1) {
-  float a[8], b[8];
+// Unscaled maxima of rows a and a+8 over a 64-key half (the four threads of a
+// row combine through shuffles).
+__device__ __forceinline__ void half_row_max(const uint32_t (&r)[32], float& x0, float& x1) {
+  float a[4], b[4];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
+  for (int j = 0; j < 4; ++j) {
     a[j] = fmaxf(fmaxf(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1])),
-                 fmaxf(__uint_as_float(r[4 * j + 32]), __uint_as_float(r[4 * j + 33])));
+                 fmaxf(__uint_as_float(r[4 * j + 16]), __uint_as_float(r[4 * j + 17])));
     b[j] = fmaxf(fmaxf(__uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])),
-                 fmaxf(__uint_as_float(r[4 * j + 34]), __uint_as_float(r[4 * j + 35])));
+                 fmaxf(__uint_as_float(r[4 * j + 18]), __uint_as_float(r[4 * j + 19])));
   }
-#pragma unroll
-  for (int w = 4; w >= 1; w >>= 1)
-#pragma unroll
-    for (int j = 0; j < w; ++j) {
-      a[j] = fmaxf(a[j], a[j + w]);
-      b[j] = fmaxf(b[j], b[j + w]);
-    }
+  a[0] = fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3]));
+  b[0] = fmaxf(fmaxf(b[0], b[1]), fmaxf(b[2], b[3]));
   x0 = fmaxf(a[0], __shfl_xor_sync(0xffffffffu, a[0], 1));
   x1 = fmaxf(b[0], __shfl_xor_sync(0xffffffffu, b[0], 1));
   x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, 2));
@@ -210,33 +206,40 @@ struct Layout {
   static constexpr int NH = D / 64;              // 128-byte column groups of a row
   static constexpr int Q_BYTES = 64 * D * 2;     // one query cube
   static constexpr int KV_BYTES = 128 * D * 2;   // two KV cubes
-  static constexpr int OFF_Q = 0;                                 // Q[stream][2]
-  static constexpr int OFF_K = OFF_Q + 4 * Q_BYTES;               // K[stream]
-  static constexpr int OFF_V = OFF_K + 2 * KV_BYTES;              // V[stream]
-  static constexpr int OFF_STAGE = OFF_V + 2 * KV_BYTES;          // output staging, 64 x D bf16
+  static constexpr int OFF_Q = 0;                                 // Q[2]
+  static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;               // K ring
+  static constexpr int OFF_V = OFF_K + kKStages * KV_BYTES;       // V ring
+  static constexpr int OFF_STAGE = OFF_V + kVStages * KV_BYTES;   // output staging, 64 x D bf16
   static constexpr int TILE_BYTES = OFF_STAGE + 64 * D * 2;
   static constexpr int SMEM_BYTES = TILE_BYTES + 1024;            // + alignment slack
 };
 
 struct __align__(8) Bars {
-  uint64_t k_full[2], k_empty[2];  // [stream]: K of a step in smem / consumed
-  uint64_t v_full[2], v_empty[2];  // [stream]: V of a step in smem / consumed
-  uint64_t q_full[2][2];   // [stream][buffer]: Q of an item in smem (TMA)
-  uint64_t s_full[2];      // MMA -> softmax of stream s: S of a step (commit)
-  uint64_t p_full[2];      // softmax -> MMA: P of a step in TMEM (count 4)
-  uint64_t l_full[2][2];   // softmax -> epilogue: 1/l of an item (count 4)
-  uint64_t o_full[2];      // MMA -> epilogue: last O step of an item (commit)
-  uint64_t o_empty[2];     // epilogue -> MMA: O read out (count 4)
+  uint64_t k_full[kKStages], k_empty[kKStages];
+  uint64_t v_full[kVStages], v_empty[kVStages];
+  uint64_t q_full[2];   // Q of item is in smem buffer is % 2 (TMA)
+  uint64_t s_full[2];   // S issuer -> softmax: S of step j in buffer j % 2 (commit)
+  uint64_t p_full[2];   // softmax -> O issuer: P of step j in buffer j % 2 (count 8)
+  uint64_t sp_free[2];  // O issuer -> S issuer, softmax: O of step j complete (commit)
+  uint64_t l_full[2];   // softmax -> epilogue: row sums of item is in buffer is % 2 (count 8)
+  uint64_t o_full[2];   // O issuer -> epilogue: O of item is complete (commit)
+  uint64_t o_empty[2];  // epilogue -> O issuer: O buffer is % 2 read out (count 4)
   uint64_t drain[2], stall;
+};
+
+// Gates and coarse output of one item, prefetched by the epilogue.
+struct alignas(16) Pre {
+  float gc[64], gf[64];  // per in-cube slot
+  float oc[128];         // coarse output row (D values)
 };
 
 struct alignas(16) Shared {
   Bars bar;
   uint32_t tmem_base;
   int abort_flag;
-  int issue_lock;                     // held by an MMA issuer while it enqueues a block
-  int epi_pick;                       // stream whose item the epilogue handles next
-  alignas(16) float inv_l[2][2][64];  // [stream][item parity][row]
+  alignas(16) float xmax[2][64];      // [key half][row]: half-row maxima on the rescale path
+  alignas(16) float lpart[2][2][64];  // [item parity][key half][row]: row sums of an item
+  Pre pre[2];                         // [item parity]
 };
 
 struct Waiter {
@@ -260,22 +263,6 @@ struct Waiter {
       }
     }
   }
-  // Bounded acquisition of a shared-memory spin lock; false on timeout or abort.
-  __device__ __forceinline__ bool acquire(int* lock) const {
-    if (atomicCAS(lock, 0, 1) == 0) return true;
-    const uint64_t t0 = globaltimer_ns();
-    while (true) {
-#pragma unroll 1
-      for (int i = 0; i < 64; ++i)
-        if (atomicCAS(lock, 0, 1) == 0) return true;
-      if (*(volatile int*)&sh->abort_flag) return false;
-      if (globaltimer_ns() - t0 > limit) {
-        *(volatile int*)&sh->abort_flag = 1;
-        atomicOr(err, kErrTimeout);
-        return false;
-      }
-    }
-  }
   // Bounded wait that ignores the abort flag (used while draining).
   __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) const {
     mbar_wait(bar, parity, limit);
@@ -288,14 +275,14 @@ __device__ __forceinline__ int raw_count(const FineParams& p, int item) {
   return p.cnt ? p.cnt[item] : p.kcap;
 }
 
-// Position of one stream in its own sequence of steps. The count of the
-// stream's next item is loaded one item ahead, so no role stalls on it at an
-// item boundary.
+// Position in the CTA's sequence of steps (items blockIdx.x + is * gridDim.x).
+// The count of the next item is loaded one item ahead, so no role stalls on
+// it at an item boundary.
 struct Cursor {
-  int is;      // item index within the stream
+  int is;      // item index within the CTA
   int item;    // global item index
   int n;       // selected cubes of the item
-  int n_next;  // raw count of the stream's next item
+  int n_next;  // raw count of the next item
   int t;       // step within the item
   int ntiles;  // steps of the item
   bool live;
@@ -312,21 +299,36 @@ __device__ __forceinline__ void cursor_enter(const FineParams& p, Cursor& c, int
   c.t = 0;
   c.ntiles = (c.n + 1) >> 1;
 }
-__device__ __forceinline__ void cursor_init(const FineParams& p, Cursor& c, int s) {
+__device__ __forceinline__ void cursor_init(const FineParams& p, Cursor& c) {
   c.is = 0;
-  c.item = blockIdx.x + s * gridDim.x;
+  c.item = blockIdx.x;
   c.bad = false;
   const int n0 = raw_count(p, c.item);
-  c.n_next = raw_count(p, c.item + 2 * gridDim.x);
+  c.n_next = raw_count(p, c.item + gridDim.x);
   cursor_enter(p, c, n0);
 }
 __device__ __forceinline__ void cursor_next(const FineParams& p, Cursor& c) {
   if (++c.t < c.ntiles) return;
   c.is += 1;
-  c.item += 2 * gridDim.x;
+  c.item += gridDim.x;
   const int n_raw = c.n_next;
-  c.n_next = raw_count(p, c.item + 2 * gridDim.x);
+  c.n_next = raw_count(p, c.item + gridDim.x);
   cursor_enter(p, c, n_raw);
+}
+
+// Rows a and a+8 of a 64-column O block scaled by a0 and a1 (one warp).
+__device__ __forceinline__ void rescale_o64(uint32_t taddr, float a0, float a1) {
+  uint32_t o[32];
+  ld_16x256b_x8(taddr, o);
+  tmem_wait_ld();
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    o[4 * e] = __float_as_uint(__uint_as_float(o[4 * e]) * a0);
+    o[4 * e + 1] = __float_as_uint(__uint_as_float(o[4 * e + 1]) * a0);
+    o[4 * e + 2] = __float_as_uint(__uint_as_float(o[4 * e + 2]) * a1);
+    o[4 * e + 3] = __float_as_uint(__uint_as_float(o[4 * e + 3]) * a1);
+  }
+  st_16x256b_x8(taddr, o);
 }
 
 template <int D>
@@ -341,30 +343,33 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
   const int C = p.C;
 
   if (tid == 0) {
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&B.k_full[s], 1);
-      mbar_init(&B.k_empty[s], 1);
-      mbar_init(&B.v_full[s], 1);
-      mbar_init(&B.v_empty[s], 1);
-      mbar_init(&B.drain[s], 1);
-      for (int b = 0; b < 2; ++b) {
-        mbar_init(&B.q_full[s][b], 1);
-        mbar_init(&B.l_full[s][b], 4);
-      }
-      mbar_init(&B.s_full[s], 1);
-      mbar_init(&B.p_full[s], 4);
-      mbar_init(&B.o_full[s], 1);
-      mbar_init(&B.o_empty[s], 4);
+    for (int i = 0; i < kKStages; ++i) {
+      mbar_init(&B.k_full[i], 1);
+      mbar_init(&B.k_empty[i], 1);
+    }
+    for (int i = 0; i < kVStages; ++i) {
+      mbar_init(&B.v_full[i], 1);
+      mbar_init(&B.v_empty[i], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&B.q_full[b], 1);
+      mbar_init(&B.s_full[b], 1);
+      mbar_init(&B.p_full[b], 8);
+      mbar_init(&B.sp_free[b], 1);
+      mbar_init(&B.l_full[b], 8);
+      mbar_init(&B.o_full[b], 1);
+      mbar_init(&B.o_empty[b], 4);
+      mbar_init(&B.drain[b], 1);
     }
     mbar_init(&B.stall, 1);
     sh.abort_flag = 0;
-    sh.issue_lock = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&p.tm_q);
     prefetch_tmap(&p.tm_k);
     prefetch_tmap(&p.tm_v);
+    if (p.out) prefetch_tmap(&p.tm_out);
   }
   if (warp == 2) {
     tmem_alloc(&sh.tmem_base, kTmemCols);
@@ -376,14 +381,16 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
   const uint32_t tmem = sh.tmem_base;
 
   if (warp == 0 || warp == 1) {
-    // ------------------------------------------------------------ K / V producer of stream s
+    // ------------------------------------------------------------ K (warp 0) / V (warp 1) producer
     regs_dec<72>();
-    const int s = warp;
-    uint8_t* kbuf = tiles + L::OFF_K + s * L::KV_BYTES;
-    uint8_t* vbuf = tiles + L::OFF_V + s * L::KV_BYTES;
+    const bool is_k = (warp == 0);
+    const int stages = is_k ? kKStages : kVStages;
+    uint64_t* full = is_k ? B.k_full : B.v_full;
+    uint64_t* empty = is_k ? B.k_empty : B.v_empty;
+    uint8_t* ring = tiles + (is_k ? L::OFF_K : L::OFF_V);
+    const CUtensorMap* tm = is_k ? &p.tm_k : &p.tm_v;
     bool bad = false, aborted = false;
-    int g = 0;                   // steps issued
-    int k_armed = 0, v_armed = 0;  // copies armed on k_full / v_full (lane 0)
+    int g = 0;  // steps armed
     // Cube ids of a step: lanes 0 and 1 load them; -1 if absent.
     auto fetch = [&](const Cursor& c) -> int {
       int cid = -1;
@@ -394,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
       return cid;
     };
     Cursor c;
-    cursor_init(p, c, s);
+    cursor_init(p, c);
     int cid = fetch(c);
     while (c.live) {
       Cursor nx = c;  // look one step ahead so the id loads overlap this step
@@ -408,26 +415,17 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
         ca = ca < 0 || ca >= C ? 0 : ca;
         cb = cb < 0 || cb >= C ? 0 : cb;
       }
-      const int row_a = (c.item / C * C + ca) * 64, row_b = (c.item / C * C + cb) * 64;
+      const int base_row = c.item / C * C;
       if (lane == 0) {
-        if (g >= 1 && !W.wait(&B.k_empty[s], (g - 1) & 1)) aborted = true;
+        const int slot = g % stages;
+        if (g >= stages && !W.wait(&empty[slot], ((g / stages) - 1) & 1)) aborted = true;
         if (!aborted) {
-          mbar_arrive_expect_tx(&B.k_full[s], L::KV_BYTES);
-          ++k_armed;
+          mbar_arrive_expect_tx(&full[slot], L::KV_BYTES);
+          uint8_t* dst = ring + slot * L::KV_BYTES;
 #pragma unroll
           for (int h = 0; h < L::NH; ++h) {
-            tma_load_2d(kbuf + h * 16384, &p.tm_k, &B.k_full[s], 64 * h, row_a);
-            tma_load_2d(kbuf + h * 16384 + 8192, &p.tm_k, &B.k_full[s], 64 * h, row_b);
-          }
-        }
-        if (!aborted && g >= 1 && !W.wait(&B.v_empty[s], (g - 1) & 1)) aborted = true;
-        if (!aborted) {
-          mbar_arrive_expect_tx(&B.v_full[s], L::KV_BYTES);
-          ++v_armed;
-#pragma unroll
-          for (int h = 0; h < L::NH; ++h) {
-            tma_load_2d(vbuf + h * 16384, &p.tm_v, &B.v_full[s], 64 * h, row_a);
-            tma_load_2d(vbuf + h * 16384 + 8192, &p.tm_v, &B.v_full[s], 64 * h, row_b);
+            tma_load_2d(dst + h * 16384, tm, &full[slot], 64 * h, (base_row + ca) * 64);
+            tma_load_2d(dst + h * 16384 + 8192, tm, &full[slot], 64 * h, (base_row + cb) * 64);
           }
         }
       }
@@ -437,177 +435,177 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
       c = nx;
       cid = cid_next;
     }
-    if ((bad || c.bad) && lane == 0) atomicOr(p.err, kErrBadIndex);
+    if (is_k && (bad || c.bad) && lane == 0) atomicOr(p.err, kErrBadIndex);
     // Drain: phases complete in order, so waiting for the last armed phase of
-    // each barrier covers every copy this warp issued.
-    if (lane == 0 && k_armed > 0) W.drain_wait(&B.k_full[s], (k_armed - 1) & 1);
-    if (lane == 0 && v_armed > 0) W.drain_wait(&B.v_full[s], (v_armed - 1) & 1);
-  } else if (warp == 2 || warp == 3) {
-    // ------------------------------------------------------------ MMA issuer of stream s
+    // each slot covers every copy this warp issued.
+    if (lane == 0)
+      for (int slot = 0; slot < stages && slot < g; ++slot) {
+        const int uses = (g - 1 - slot) / stages + 1;
+        W.drain_wait(&full[slot], (uses - 1) & 1);
+      }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ S issuer
     regs_dec<72>();
     if (lane == 0) {
-      const int s = warp - 2;
       constexpr uint32_t idesc_s = idesc_bf16_f32(64, 128, false, false);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(64, D, false, true);
-      const uint64_t qdesc0 = sdesc_sw128(smem_u32(tiles + L::OFF_Q + 2 * s * L::Q_BYTES), 16, 1024);
-      const uint64_t kdesc = sdesc_sw128(smem_u32(tiles + L::OFF_K + s * L::KV_BYTES), 16, 1024);
-      const uint64_t vdesc = sdesc_sw128(smem_u32(tiles + L::OFF_V + s * L::KV_BYTES), 16384, 1024);
-      const uint32_t tS = tmem + kColSP + 128u * s, tO = tmem + kColO + 128u * s;
+      const uint64_t qdesc0 = sdesc_sw128(smem_u32(tiles + L::OFF_Q), 16, 1024);
+      const uint64_t kdesc0 = sdesc_sw128(smem_u32(tiles + L::OFF_K), 16, 1024);
       bool aborted = false, issued_any = false;
       if (p.debug_stall && !W.wait(&B.stall, 0)) aborted = true;
       Cursor c;
-      cursor_init(p, c, s);
-      int j = 0;  // steps of this stream
-      // Each block ([S(0)], then [O(j), S(j+1)]) is enqueued under the issue
-      // lock once all its operands are ready, so the two streams' blocks reach
-      // the tensor core whole and in turn: one stream's S completes a block
-      // ahead of the other's and the two softmax groups run staggered instead
-      // of contending for the same units.
-      bool ok = !aborted && c.live;
-      if (ok) ok = W.wait(&B.q_full[s][0], 0) && W.wait(&B.k_full[s], 0) && W.acquire(&sh.issue_lock);
-      if (ok) {
-        tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k)
-          mma_bf16_ss(tS, qdesc0 + (uint64_t)(((k >> 2) * 8192 + (k & 3) * 32) >> 4),
-                      kdesc + (uint64_t)(((k >> 2) * 16384 + (k & 3) * 32) >> 4), idesc_s, k > 0 ? 1u : 0u);
-        mma_commit(&B.k_empty[s]);
-        mma_commit(&B.s_full[s]);
-        atomicExch(&sh.issue_lock, 0);
-        issued_any = true;
-      } else if (c.live) {
-        aborted = true;
-      }
+      cursor_init(p, c);
+      int j = 0;  // steps of the CTA
       while (!aborted && c.live) {
-        // O of step j (P in TMEM, V in smem), then S of step j + 1.
-        const bool first = (c.t == 0), last = (c.t == c.ntiles - 1);
-        const int is = c.is;
-        Cursor nx = c;
-        cursor_next(p, nx);
-        const int qb = nx.is & 1;
-        if (!W.wait(&B.v_full[s], j & 1) || !W.wait(&B.p_full[s], j & 1) ||
-            (first && is >= 1 && !W.wait(&B.o_empty[s], (is - 1) & 1)) ||
-            (nx.live && nx.t == 0 && !W.wait(&B.q_full[s][qb], (nx.is >> 1) & 1)) ||
-            (nx.live && !W.wait(&B.k_full[s], (j + 1) & 1)) || !W.acquire(&sh.issue_lock)) {
+        const int b = j & 1, ks = j % kKStages;
+        // Buffer b is free once O of step j - 2 (which read its P) completed.
+        if ((j >= 2 && !W.wait(&B.sp_free[b], ((j >> 1) - 1) & 1)) ||
+            (c.t == 0 && !W.wait(&B.q_full[c.is & 1], (c.is >> 1) & 1)) ||
+            !W.wait(&B.k_full[ks], (j / kKStages) & 1)) {
           aborted = true;
           break;
         }
         tc_fence_after();
+        const uint64_t qd = qdesc0 + (uint64_t)(((c.is & 1) * L::Q_BYTES) >> 4);
+        const uint64_t kd = kdesc0 + (uint64_t)((ks * L::KV_BYTES) >> 4);
 #pragma unroll
-        for (int k = 0; k < 8; ++k)  // 8 steps of 16 keys; P step k = 8 TMEM columns
-          mma_bf16_ts(tO, tS + 8u * k, vdesc + (uint64_t)((k * 2048) >> 4), idesc_o, (first && k == 0) ? 0u : 1u);
-        mma_commit(&B.v_empty[s]);
-        if (last) mma_commit(&B.o_full[s]);
-        if (nx.live) {
-          const uint64_t qd = qdesc0 + (uint64_t)((qb * L::Q_BYTES) >> 4);
-#pragma unroll
-          for (int k = 0; k < D / 16; ++k)  // steps of 16 along D
-            mma_bf16_ss(tS, qd + (uint64_t)(((k >> 2) * 8192 + (k & 3) * 32) >> 4),
-                        kdesc + (uint64_t)(((k >> 2) * 16384 + (k & 3) * 32) >> 4), idesc_s, k > 0 ? 1u : 0u);
-          mma_commit(&B.k_empty[s]);
-          mma_commit(&B.s_full[s]);
-        }
-        atomicExch(&sh.issue_lock, 0);
+        for (int k = 0; k < D / 16; ++k)  // steps of 16 along D
+          mma_bf16_ss(tmem + kColSP + 128u * b, qd + (uint64_t)(((k >> 2) * 8192 + (k & 3) * 32) >> 4),
+                      kd + (uint64_t)(((k >> 2) * 16384 + (k & 3) * 32) >> 4), idesc_s, k > 0 ? 1u : 0u);
+        mma_commit(&B.k_empty[ks]);
+        mma_commit(&B.s_full[b]);
+        issued_any = true;
         ++j;
-        c = nx;
+        cursor_next(p, c);
       }
       // Drain: every MMA issued by this thread completes before TMEM is released.
       if (issued_any) {
-        mma_commit(&B.drain[s]);
-        W.drain_wait(&B.drain[s], 0);
+        mma_commit(&B.drain[0]);
+        W.drain_wait(&B.drain[0], 0);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ O issuer
+    regs_dec<72>();
+    if (lane == 0) {
+      constexpr uint32_t idesc_o = idesc_bf16_f32(64, D, false, true);
+      const uint64_t vdesc0 = sdesc_sw128(smem_u32(tiles + L::OFF_V), 16384, 1024);
+      bool aborted = false, issued_any = false;
+      Cursor c;
+      cursor_init(p, c);
+      int j = 0;
+      while (!aborted && c.live) {
+        const int b = j & 1, vs = j % kVStages, ob = c.is & 1;
+        const bool first = (c.t == 0), last = (c.t == c.ntiles - 1);
+        if ((first && c.is >= 2 && !W.wait(&B.o_empty[ob], ((c.is >> 1) - 1) & 1)) ||
+            !W.wait(&B.v_full[vs], (j / kVStages) & 1) || !W.wait(&B.p_full[b], (j >> 1) & 1)) {
+          aborted = true;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t vd = vdesc0 + (uint64_t)((vs * L::KV_BYTES) >> 4);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)  // 8 steps of 16 keys; P step k = 8 TMEM columns
+          mma_bf16_ts(tmem + kColO + 128u * ob, tmem + kColSP + 128u * b + 8u * k, vd + (uint64_t)((k * 2048) >> 4),
+                      idesc_o, (first && k == 0) ? 0u : 1u);
+        mma_commit(&B.v_empty[vs]);
+        mma_commit(&B.sp_free[b]);
+        if (last) mma_commit(&B.o_full[ob]);
+        issued_any = true;
+        ++j;
+        cursor_next(p, c);
+      }
+      if (issued_any) {
+        mma_commit(&B.drain[1]);
+        W.drain_wait(&B.drain[1], 0);
       }
     }
     __syncwarp();
   } else if (warp >= 4 && warp < 12) {
-    // ------------------------------------------------------------ softmax (stream s)
+    // ------------------------------------------------------------ softmax
     regs_inc<152>();
-    const int s = (warp - 4) >> 2;
-    const int quarter = warp & 3;
+    const int quarter = warp & 3, hf = (warp - 4) >> 2;  // lane quarter, key half
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    const uint32_t tSP = tmem + kColSP + 128u * s + lane_base;
-    const uint32_t tO = tmem + kColO + 128u * s + lane_base;
+    const int ra = quarter * 16 + (lane >> 2);  // rows ra and ra + 8
     const float scale = p.scale_log2;
-    int tc = 0;  // steps processed by this stream
+    int j = 0;  // steps of the CTA
     Cursor c;
-    cursor_init(p, c, s);
+    cursor_init(p, c);
     while (c.live) {
-      const int n = c.n, ntiles = c.ntiles, is = c.is;
-      float m0 = -INFINITY, m1 = -INFINITY;  // reference max (scaled) of rows a and a+8
+      const int n = c.n, ntiles = c.ntiles, ob = c.is & 1;
+      float m0 = -INFINITY, m1 = -INFINITY;  // reference max (scaled) of rows ra and ra+8
       float l0 = 0.f, l1 = 0.f;              // this thread's share of the row sums
-      for (int t = 0; t < ntiles; ++t, ++tc) {
-        W.wait(&B.s_full[s], tc & 1);
+      for (int t = 0; t < ntiles; ++t, ++j) {
+        const int b = j & 1;
+        const uint32_t tS = tmem + kColSP + 128u * b + lane_base;
+        W.wait(&B.s_full[b], (j >> 1) & 1);
         tc_fence_after();
-        uint32_t r[64];
-        ld_16x256b_x16(tSP, r);
+        uint32_t r[32];
+        ld_16x256b_x8(tS + 64u * hf, r);
         tmem_wait_ld();
-        const bool tail = (2 * t + 1 >= n);
-        if (tail) {
-          // Odd tail: keys 64..127 (the repeated cube) do not take part.
+        // Odd tail: keys 64..127 (the repeated cube) do not take part.
+        const bool masked = hf == 1 && (2 * t + 1 >= n);
+        if (masked) {
 #pragma unroll
-          for (int e = 32; e < 64; ++e) r[e] = __float_as_uint(-INFINITY);
+          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(-INFINITY);
         }
         // Optimistic pass with the current reference max. A thread's partial
         // row sum exceeds 2^8 whenever one of its scores exceeds the reference
         // by more than 2^8 (and when the reference is still -inf), so only then
-        // is the exact row max needed.
-        uint32_t pk[32];
+        // are the exact row maxima needed.
+        uint32_t pk[16];
         float s0, s1;
-        if (tail) exp_pack<false>(r, scale, m0, m1, pk, s0, s1);
+        if (masked) exp_pack<false>(r, scale, m0, m1, pk, s0, s1);
         else exp_pack<true>(r, scale, m0, m1, pk, s0, s1);
-        if (__any_sync(0xffffffffu, !(s0 <= 256.f) || !(s1 <= 256.f))) {
+        if (pair_any(quarter, !(s0 <= 256.f) || !(s1 <= 256.f))) {
           float x0, x1;
-          row_max(r, x0, x1);
-          x0 *= scale;
-          x1 *= scale;
-          // Lazy reference update per row.
+          half_row_max(r, x0, x1);
+          if ((lane & 3) == 0) {
+            sh.xmax[hf][ra] = x0;
+            sh.xmax[hf][ra + 8] = x1;
+          }
+          pair_sync(quarter);
+          x0 = fmaxf(sh.xmax[0][ra], sh.xmax[1][ra]) * scale;
+          x1 = fmaxf(sh.xmax[0][ra + 8], sh.xmax[1][ra + 8]) * scale;
+          pair_sync(quarter);
+          // Lazy reference update per row (identical in both warps of the pair).
           float a0 = 1.f, a1 = 1.f;
           const bool u0 = x0 > m0 + 8.0f, u1 = x1 > m1 + 8.0f;
           if (u0) { a0 = fast_exp2(m0 - x0); m0 = x0; l0 *= a0; }
           if (u1) { a1 = fast_exp2(m1 - x1); m1 = x1; l1 *= a1; }
           if (__any_sync(0xffffffffu, u0 || u1)) {
-            if (t > 0) {
-              // O holds steps < t of this item (their MMAs completed before
-              // this step's S): rescale the rows in place, 64 columns at a time.
-#pragma unroll
-              for (int h = 0; h < D / 64; ++h) {
-                uint32_t o[32];
-                ld_16x256b_x8(tO + 64u * h, o);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                  o[4 * e] = __float_as_uint(__uint_as_float(o[4 * e]) * a0);
-                  o[4 * e + 1] = __float_as_uint(__uint_as_float(o[4 * e + 1]) * a0);
-                  o[4 * e + 2] = __float_as_uint(__uint_as_float(o[4 * e + 2]) * a1);
-                  o[4 * e + 3] = __float_as_uint(__uint_as_float(o[4 * e + 3]) * a1);
-                }
-                st_16x256b_x8(tO + 64u * h, o);
-              }
+            if (t > 0 && (D == 128 || hf == 0)) {
+              // O holds steps < t of this item: wait for the last of them to
+              // complete, then rescale this warp's 64 columns of the rows
+              // (D = 64: the first warp of the pair takes all of them).
+              W.wait(&B.sp_free[(j - 1) & 1], ((j - 1) >> 1) & 1);
+              tc_fence_after();
+              rescale_o64(tmem + kColO + 128u * ob + lane_base + (D == 128 ? 64u * hf : 0u), a0, a1);
               tmem_wait_st();
             }
-            if (tail) exp_pack<false>(r, scale, m0, m1, pk, s0, s1);
+            if (masked) exp_pack<false>(r, scale, m0, m1, pk, s0, s1);
             else exp_pack<true>(r, scale, m0, m1, pk, s0, s1);
           }
         }
         l0 += s0;
         l1 += s1;
-        st_16x128b_x16(tSP, pk);
+        st_16x128b_x8(tS + 32u * hf, pk);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&B.p_full[s]);
+        if (lane == 0) mbar_arrive(&B.p_full[b]);
       }
-      // Row sums of the item -> 1/l for the epilogue.
+      // Row sums of the item (this key half) -> the epilogue.
       l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
       l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
       l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
       l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
       if ((lane & 3) == 0) {
-        const int row = quarter * 16 + (lane >> 2);
-        sh.inv_l[s][is & 1][row] = 1.0f / l0;
-        sh.inv_l[s][is & 1][row + 8] = 1.0f / l1;
+        sh.lpart[ob][hf][ra] = l0;
+        sh.lpart[ob][hf][ra + 8] = l1;
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&B.l_full[s][is & 1]);
+      if (lane == 0) mbar_arrive(&B.l_full[ob]);
       c.t = c.ntiles - 1;
       cursor_next(p, c);
     }
@@ -621,118 +619,125 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
     const int est = tid - 384;                  // 0..127 within the epilogue group
     uint8_t* stage = tiles + L::OFF_STAGE;
     const int Hc = p.H >> 2, Wc = p.W >> 2;
-    int qloads[2][2] = {{0, 0}, {0, 0}};
-    // Q of item `is` of stream s -> smem buffer [s][is & 1] (TMA, one thread).
-    auto load_q = [&](int s, int is) {
-      const int item = blockIdx.x + (s + 2 * is) * gridDim.x;
+    int qloads0 = 0, qloads1 = 0;
+    // Q of item `is` -> smem buffer is & 1 (TMA, one thread).
+    auto load_q = [&](int is) {
+      const int item = blockIdx.x + is * gridDim.x;
       if (item >= p.n_items) return;
       const int b = is & 1;
-      ++qloads[s][b];
+      if (b == 0) ++qloads0; else ++qloads1;
       if (est == 0) {
-        uint8_t* dst = tiles + L::OFF_Q + (2 * s + b) * L::Q_BYTES;
-        mbar_arrive_expect_tx(&B.q_full[s][b], L::Q_BYTES);
+        uint8_t* dst = tiles + L::OFF_Q + b * L::Q_BYTES;
+        mbar_arrive_expect_tx(&B.q_full[b], L::Q_BYTES);
 #pragma unroll
-        for (int h = 0; h < L::NH; ++h) tma_load_2d(dst + h * 8192, &p.tm_q, &B.q_full[s][b], 64 * h, item * 64);
+        for (int h = 0; h < L::NH; ++h) tma_load_2d(dst + h * 8192, &p.tm_q, &B.q_full[b], 64 * h, item * 64);
       }
     };
-    for (int s = 0; s < 2; ++s) {
-      load_q(s, 0);
-      load_q(s, 1);
-    }
-    // Items are finished in whatever order the two streams complete them (a
-    // fixed order would let a long item of one stream hold back the other
-    // stream's O buffer). Thread 0 of the group picks the stream; the group
-    // follows through shared memory.
-    int next_is[2] = {0, 0};
-    while (true) {
-      const bool live0 = blockIdx.x + (2 * next_is[0]) * gridDim.x < p.n_items;
-      const bool live1 = blockIdx.x + (1 + 2 * next_is[1]) * gridDim.x < p.n_items;
-      if (!live0 && !live1) break;
-      if (est == 0) {
-        int pick = live0 ? 0 : 1;
-        if (live0 && live1) {
-          const uint64_t t0 = globaltimer_ns();
-          pick = -1;
-          while (pick < 0) {
-            if (mbar_try_wait(&B.o_full[0], next_is[0] & 1)) pick = 0;
-            else if (mbar_try_wait(&B.o_full[1], next_is[1] & 1)) pick = 1;
-            else if (*(volatile int*)&sh.abort_flag || globaltimer_ns() - t0 > p.wait_ns) pick = 0;
-          }
+    // Gates (16 runs of 4 raster tokens per gate array) and the coarse output
+    // row of item `is` -> sh.pre[is & 1]; one cp.async group per call on
+    // every thread, so groups stay in the same order everywhere.
+    auto prefetch = [&](int is) {
+      const int item = blockIdx.x + is * gridDim.x;
+      if (item < p.n_items && est < 32 + D / 4) {
+        const int bh = item / C, ci = item - bh * C;
+        Pre& pr = sh.pre[is & 1];
+        if (est < 32) {
+          const int run = est & 15;  // in-cube slots 4 run .. 4 run + 3: t = run / 4, h = run % 4
+          const int ct = ci / (Hc * Wc), ch = (ci / Wc) % Hc, cw = ci % Wc;
+          const int tok = ((4 * ct + (run >> 2)) * p.H + 4 * ch + (run & 3)) * p.W + 4 * cw;
+          const float* g = (est < 16 ? p.gate_c : p.gate_f) + (size_t)bh * p.N + tok;
+          cp_async16(est < 16 ? &pr.gc[4 * run] : &pr.gf[4 * run], g);
+        } else {
+          const int e = est - 32;
+          cp_async16(&pr.oc[4 * e], p.oc + ((size_t)bh * C + ci) * D + 4 * e);
         }
-        sh.epi_pick = pick;
       }
-      epi_sync();
-      const int s = sh.epi_pick;
-      const int is = next_is[s]++;
-      const int item = blockIdx.x + (s + 2 * is) * gridDim.x;
+      cp_async_commit();
+    };
+    load_q(0);
+    load_q(1);
+    prefetch(0);
+    for (int is = 0; blockIdx.x + is * gridDim.x < p.n_items; ++is) {
+      const int item = blockIdx.x + is * gridDim.x;
       const int bh = item / C, ci = item - bh * C;
-      // raster token of the cube's first row; row q adds ((q>>4)*H + (q>>2&3))*W + (q&3)
       const int ct = ci / (Hc * Wc), ch = (ci / Wc) % Hc, cw = ci % Wc;
-      const int tok_base = ((4 * ct) * p.H + 4 * ch) * p.W + 4 * cw;
-      auto tok_of = [&](int q) { return tok_base + ((q >> 4) * p.H + ((q >> 2) & 3)) * p.W + (q & 3); };
-      const int tok0 = tok_of(ra), tok1 = tok_of(ra + 8);
-      const float gc0 = p.gate_c[(size_t)bh * p.N + tok0], gf0 = p.gate_f[(size_t)bh * p.N + tok0];
-      const float gc1 = p.gate_c[(size_t)bh * p.N + tok1], gf1 = p.gate_f[(size_t)bh * p.N + tok1];
-      const float* ocrow = p.oc + ((size_t)bh * C + ci) * D;
-      W.wait(&B.l_full[s][is & 1], (is >> 1) & 1);
-      const float il0 = sh.inv_l[s][is & 1][ra], il1 = sh.inv_l[s][is & 1][ra + 8];
-      W.wait(&B.o_full[s], is & 1);
+      const int ob = is & 1;
+      prefetch(is + 1);
+      W.wait(&B.l_full[ob], (is >> 1) & 1);
+      const float il0 = 1.0f / (sh.lpart[ob][0][ra] + sh.lpart[ob][1][ra]);
+      const float il1 = 1.0f / (sh.lpart[ob][0][ra + 8] + sh.lpart[ob][1][ra + 8]);
+      W.wait(&B.o_full[ob], (is >> 1) & 1);
       tc_fence_after();
       float o[2 * D / 4];
 #pragma unroll
       for (int h = 0; h < D / 64; ++h) {
         uint32_t r[32];
-        ld_16x256b_x8(tmem + kColO + 128u * s + 64u * h + lane_base, r);
+        ld_16x256b_x8(tmem + kColO + 128u * ob + 64u * h + lane_base, r);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) o[32 * h + j] = __uint_as_float(r[j]);
+        for (int jj = 0; jj < 32; ++jj) o[32 * h + jj] = __uint_as_float(r[jj]);
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&B.o_empty[s]);
-      // All S steps of this item completed: its Q buffer takes the stream's item after next.
-      load_q(s, is + 2);
+      if (lane == 0) mbar_arrive(&B.o_empty[ob]);
+      // All S steps of this item completed: its Q buffer takes item is + 2.
+      load_q(is + 2);
+      cp_async_wait<1>();               // this item's gates and coarse row (older group) landed
+      if (est == 0) bulk_wait_read0();  // the previous item's output stores have read the staging tile
+      epi_sync();
+      const Pre& pr = sh.pre[ob];
+      const float gc0 = pr.gc[ra], gf0 = pr.gf[ra], gc1 = pr.gc[ra + 8], gf1 = pr.gf[ra + 8];
       // o[4j..4j+3] = (row ra: d, d+1; row ra+8: d, d+1), d = 8j + 2 tq
       if (p.out_fine) {
+        // raster token of in-cube slot q: ((4ct + q/16) H + 4ch + (q/4)%4) W + 4cw + q%4
+        auto tok_of = [&](int q) { return ((4 * ct + (q >> 4)) * p.H + 4 * ch + ((q >> 2) & 3)) * p.W + 4 * cw + (q & 3); };
+        const int tok0 = tok_of(ra), tok1 = tok_of(ra + 8);
 #pragma unroll
-        for (int j = 0; j < D / 8; ++j) {
-          const int d = 8 * j + 2 * tq;
+        for (int jj = 0; jj < D / 8; ++jj) {
+          const int d = 8 * jj + 2 * tq;
           *reinterpret_cast<float2*>(p.out_fine + ((size_t)bh * p.N + tok0) * D + d) =
-              make_float2(o[4 * j] * il0, o[4 * j + 1] * il0);
+              make_float2(o[4 * jj] * il0, o[4 * jj + 1] * il0);
           *reinterpret_cast<float2*>(p.out_fine + ((size_t)bh * p.N + tok1) * D + d) =
-              make_float2(o[4 * j + 2] * il1, o[4 * j + 3] * il1);
+              make_float2(o[4 * jj + 2] * il1, o[4 * jj + 3] * il1);
         }
       }
       if (p.out) {
+        // Staging tile: per 64-column group a [64 slots][128 B] block in the
+        // 128-byte swizzle of the output map (16-byte chunk c of row q at
+        // c ^ (q % 8)); rows ra and ra + 8 share q % 8.
         const float f0 = gf0 * il0, f1 = gf1 * il1;
+        const uint32_t sw = (uint32_t)(ra & 7);
 #pragma unroll
-        for (int j = 0; j < D / 8; ++j) {
-          const int d = 8 * j + 2 * tq;
-          const float2 oc = *reinterpret_cast<const float2*>(ocrow + d);
+        for (int jj = 0; jj < D / 8; ++jj) {
+          const int d = 8 * jj + 2 * tq;
+          const float2 oc = *reinterpret_cast<const float2*>(&pr.oc[d]);
           const __nv_bfloat162 h0 =
-              __floats2bfloat162_rn(fmaf(gc0, oc.x, f0 * o[4 * j]), fmaf(gc0, oc.y, f0 * o[4 * j + 1]));
+              __floats2bfloat162_rn(fmaf(gc0, oc.x, f0 * o[4 * jj]), fmaf(gc0, oc.y, f0 * o[4 * jj + 1]));
           const __nv_bfloat162 h1 =
-              __floats2bfloat162_rn(fmaf(gc1, oc.x, f1 * o[4 * j + 2]), fmaf(gc1, oc.y, f1 * o[4 * j + 3]));
-          *reinterpret_cast<__nv_bfloat162*>(stage + (ra * D + d) * 2) = h0;
-          *reinterpret_cast<__nv_bfloat162*>(stage + ((ra + 8) * D + d) * 2) = h1;
+              __floats2bfloat162_rn(fmaf(gc1, oc.x, f1 * o[4 * jj + 2]), fmaf(gc1, oc.y, f1 * o[4 * jj + 3]));
+          uint8_t* blk = stage + (jj >> 3) * 8192 + ((((uint32_t)jj & 7u) ^ sw) << 4) + 4 * tq;
+          *reinterpret_cast<__nv_bfloat162*>(blk + ra * 128) = h0;
+          *reinterpret_cast<__nv_bfloat162*>(blk + (ra + 8) * 128) = h1;
         }
+        fence_proxy_async_smem();
         epi_sync();
-        constexpr int CPR = D / 8;  // 16-byte chunks per row
+        if (est == 0) {
 #pragma unroll
-        for (int u = 0; u < (64 * CPR) / 128; ++u) {
-          const int cidx = est + 128 * u;
-          const int q = cidx / CPR, off = cidx % CPR;
-          const uint4 v = *reinterpret_cast<const uint4*>(stage + (q * D + off * 8) * 2);
-          *reinterpret_cast<uint4*>(p.out + ((size_t)bh * p.N + tok_of(q)) * D + off * 8) = v;
+          for (int h = 0; h < D / 64; ++h) tma_store_5d(&p.tm_out, stage + h * 8192, 64 * h, 4 * cw, 4 * ch, 4 * ct, bh);
+          bulk_commit();
         }
+      } else {
+        epi_sync();  // this item's gate reads are done before the buffer refills
       }
-      epi_sync();  // staging reads and the stream pick are done before the next item
     }
-    // Drain: the last Q copy of each buffer has landed (it has, unless the run aborted).
-    if (est == 0)
-      for (int s2 = 0; s2 < 2; ++s2)
-        for (int b = 0; b < 2; ++b)
-          if (qloads[s2][b] > 0) W.drain_wait(&B.q_full[s2][b], (qloads[s2][b] - 1) & 1);
+    cp_async_wait<0>();
+    // Drain: the output stores are complete and the last Q copy of each
+    // buffer has landed (it has, unless the run aborted).
+    if (est == 0) {
+      bulk_wait0();
+      if (qloads0 > 0) W.drain_wait(&B.q_full[0], (qloads0 - 1) & 1);
+      if (qloads1 > 0) W.drain_wait(&B.q_full[1], (qloads1 - 1) & 1);
+    }
   }
 
   tc_fence_before();

@@ -47,6 +47,7 @@ struct CoarseParams {
 
 struct FineParams {
   CUtensorMap tm_q, tm_k, tm_v;  // 2-D maps over the cube-major copies, rows of D bf16
+  CUtensorMap tm_out;            // 5-D map over out [BH][T][H][W][D], 64-column boxes of one cube, 128 B swizzle
   const int32_t* idx;            // [BH, C, kcap]
   const int32_t* cnt;            // [BH, C] or null (then every row has kcap ids)
   const float* oc;               // [BH, C, D]
