@@ -14,10 +14,12 @@
 //   S[64 q x 128 keys] = Q . K_pair^T     tcgen05.mma M=64, N=128 (Q, K in smem)
 //   O[64 q x D]       += P . V_pair       tcgen05.mma M=64, N=D   (P in TMEM, V in smem)
 //
-// Tensor memory holds two S/P buffers and two O accumulators, so S of step
-// j+1 runs on the tensor core while the softmax works on step j, and the
-// epilogue reads an item's O while the next item accumulates into the other
-// buffer. All eight softmax warps work on the same step: warp w handles the
+// Tensor memory holds three S/P buffers and the O accumulator: S of steps
+// j+1 and j+2 can run on the tensor core while the softmax works on step j,
+// so the chain softmax -> O MMA -> S MMA (which must wait for the O MMA that
+// read the buffer's P) spans three steps. The epilogue reads an item's O as
+// soon as its last MMA completes; the next item's first O MMA waits for that
+// read only. All eight softmax warps work on the same step: warp w handles the
 // rows of TMEM lane quarter w % 4 and the key half w / 4 (64 keys). The two
 // warps that share rows agree on the row statistics through a 64-thread
 // named barrier.
@@ -58,9 +60,10 @@ using namespace ptx;
 constexpr int kThreads = 512;
 constexpr int kKStages = 3;  // K ring depth (steps of two cubes)
 constexpr int kVStages = 2;  // V ring depth
+constexpr int kSP = 3;       // S/P buffers in tensor memory
 constexpr uint32_t kTmemCols = 512;
-// TMEM columns: S/P buffer b at 128 b, O buffer b at 256 + 128 b.
-constexpr uint32_t kColSP = 0, kColO = 256;
+// TMEM columns: S/P buffer b at 128 b, O at 384.
+constexpr uint32_t kColSP = 0, kColO = 384;
 
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
@@ -217,13 +220,13 @@ struct Layout {
 struct __align__(8) Bars {
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
-  uint64_t q_full[2];   // Q of item is in smem buffer is % 2 (TMA)
-  uint64_t s_full[2];   // S issuer -> softmax: S of step j in buffer j % 2 (commit)
-  uint64_t p_full[2];   // softmax -> O issuer: P of step j in buffer j % 2 (count 8)
-  uint64_t sp_free[2];  // O issuer -> S issuer, softmax: O of step j complete (commit)
-  uint64_t l_full[2];   // softmax -> epilogue: row sums of item is in buffer is % 2 (count 8)
-  uint64_t o_full[2];   // O issuer -> epilogue: O of item is complete (commit)
-  uint64_t o_empty[2];  // epilogue -> O issuer: O buffer is % 2 read out (count 4)
+  uint64_t q_full[2];     // Q of item is in smem buffer is % 2 (TMA)
+  uint64_t s_full[kSP];   // S issuer -> softmax: S of step j in buffer j % 3 (commit)
+  uint64_t p_full[kSP];   // softmax -> O issuer: P of step j in buffer j % 3 (count 8)
+  uint64_t sp_free[kSP];  // O issuer -> S issuer, softmax: O of step j complete (commit)
+  uint64_t l_full[2];     // softmax -> epilogue: row sums of item is in lpart[is % 2] (count 8)
+  uint64_t o_full;        // O issuer -> epilogue: O of an item complete (commit)
+  uint64_t o_empty;       // epilogue -> O issuer: O read out (count 4)
   uint64_t drain[2], stall;
 };
 
@@ -351,16 +354,18 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
       mbar_init(&B.v_full[i], 1);
       mbar_init(&B.v_empty[i], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&B.q_full[b], 1);
+    for (int b = 0; b < kSP; ++b) {
       mbar_init(&B.s_full[b], 1);
       mbar_init(&B.p_full[b], 8);
       mbar_init(&B.sp_free[b], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&B.q_full[b], 1);
       mbar_init(&B.l_full[b], 8);
-      mbar_init(&B.o_full[b], 1);
-      mbar_init(&B.o_empty[b], 4);
       mbar_init(&B.drain[b], 1);
     }
+    mbar_init(&B.o_full, 1);
+    mbar_init(&B.o_empty, 4);
     mbar_init(&B.stall, 1);
     sh.abort_flag = 0;
     fence_mbar_init();
@@ -454,11 +459,12 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
       if (p.debug_stall && !W.wait(&B.stall, 0)) aborted = true;
       Cursor c;
       cursor_init(p, c);
-      int j = 0;  // steps of the CTA
+      int j = 0;         // steps of the CTA
+      int b = 0, u = 0;  // S/P buffer of step j (j % 3) and its use count (j / 3)
       while (!aborted && c.live) {
-        const int b = j & 1, ks = j % kKStages;
-        // Buffer b is free once O of step j - 2 (which read its P) completed.
-        if ((j >= 2 && !W.wait(&B.sp_free[b], ((j >> 1) - 1) & 1)) ||
+        const int ks = j % kKStages;
+        // Buffer b is free once O of step j - 3 (which read its P) completed.
+        if ((u >= 1 && !W.wait(&B.sp_free[b], (u - 1) & 1)) ||
             (c.t == 0 && !W.wait(&B.q_full[c.is & 1], (c.is >> 1) & 1)) ||
             !W.wait(&B.k_full[ks], (j / kKStages) & 1)) {
           aborted = true;
@@ -475,6 +481,7 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
         mma_commit(&B.s_full[b]);
         issued_any = true;
         ++j;
+        if (++b == kSP) { b = 0; ++u; }
         cursor_next(p, c);
       }
       // Drain: every MMA issued by this thread completes before TMEM is released.
@@ -494,11 +501,12 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
       Cursor c;
       cursor_init(p, c);
       int j = 0;
+      int b = 0, u = 0;  // S/P buffer of step j and its use count
       while (!aborted && c.live) {
-        const int b = j & 1, vs = j % kVStages, ob = c.is & 1;
+        const int vs = j % kVStages;
         const bool first = (c.t == 0), last = (c.t == c.ntiles - 1);
-        if ((first && c.is >= 2 && !W.wait(&B.o_empty[ob], ((c.is >> 1) - 1) & 1)) ||
-            !W.wait(&B.v_full[vs], (j / kVStages) & 1) || !W.wait(&B.p_full[b], (j >> 1) & 1)) {
+        if ((first && c.is >= 1 && !W.wait(&B.o_empty, (c.is - 1) & 1)) ||
+            !W.wait(&B.v_full[vs], (j / kVStages) & 1) || !W.wait(&B.p_full[b], u & 1)) {
           aborted = true;
           break;
         }
@@ -506,13 +514,14 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
         const uint64_t vd = vdesc0 + (uint64_t)((vs * L::KV_BYTES) >> 4);
 #pragma unroll
         for (int k = 0; k < 8; ++k)  // 8 steps of 16 keys; P step k = 8 TMEM columns
-          mma_bf16_ts(tmem + kColO + 128u * ob, tmem + kColSP + 128u * b + 8u * k, vd + (uint64_t)((k * 2048) >> 4),
-                      idesc_o, (first && k == 0) ? 0u : 1u);
+          mma_bf16_ts(tmem + kColO, tmem + kColSP + 128u * b + 8u * k, vd + (uint64_t)((k * 2048) >> 4), idesc_o,
+                      (first && k == 0) ? 0u : 1u);
         mma_commit(&B.v_empty[vs]);
         mma_commit(&B.sp_free[b]);
-        if (last) mma_commit(&B.o_full[ob]);
+        if (last) mma_commit(&B.o_full);
         issued_any = true;
         ++j;
+        if (++b == kSP) { b = 0; ++u; }
         cursor_next(p, c);
       }
       if (issued_any) {
@@ -528,17 +537,16 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const int ra = quarter * 16 + (lane >> 2);  // rows ra and ra + 8
     const float scale = p.scale_log2;
-    int j = 0;  // steps of the CTA
+    int b = 0, u = 0;  // S/P buffer of the step (step % 3) and its use count (step / 3)
     Cursor c;
     cursor_init(p, c);
     while (c.live) {
       const int n = c.n, ntiles = c.ntiles, ob = c.is & 1;
       float m0 = -INFINITY, m1 = -INFINITY;  // reference max (scaled) of rows ra and ra+8
       float l0 = 0.f, l1 = 0.f;              // this thread's share of the row sums
-      for (int t = 0; t < ntiles; ++t, ++j) {
-        const int b = j & 1;
+      for (int t = 0; t < ntiles; ++t) {
         const uint32_t tS = tmem + kColSP + 128u * b + lane_base;
-        W.wait(&B.s_full[b], (j >> 1) & 1);
+        W.wait(&B.s_full[b], u & 1);
         tc_fence_after();
         uint32_t r[32];
         ld_16x256b_x8(tS + 64u * hf, r);
@@ -578,9 +586,10 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
               // O holds steps < t of this item: wait for the last of them to
               // complete, then rescale this warp's 64 columns of the rows
               // (D = 64: the first warp of the pair takes all of them).
-              W.wait(&B.sp_free[(j - 1) & 1], ((j - 1) >> 1) & 1);
+              const int pb = b == 0 ? kSP - 1 : b - 1, pu = b == 0 ? u - 1 : u;  // buffer, use of step - 1
+              W.wait(&B.sp_free[pb], pu & 1);
               tc_fence_after();
-              rescale_o64(tmem + kColO + 128u * ob + lane_base + (D == 128 ? 64u * hf : 0u), a0, a1);
+              rescale_o64(tmem + kColO + lane_base + (D == 128 ? 64u * hf : 0u), a0, a1);
               tmem_wait_st();
             }
             if (masked) exp_pack<false>(r, scale, m0, m1, pk, s0, s1);
@@ -594,6 +603,7 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&B.p_full[b]);
+        if (++b == kSP) { b = 0; ++u; }
       }
       // Row sums of the item (this key half) -> the epilogue.
       l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
@@ -666,20 +676,20 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
       W.wait(&B.l_full[ob], (is >> 1) & 1);
       const float il0 = 1.0f / (sh.lpart[ob][0][ra] + sh.lpart[ob][1][ra]);
       const float il1 = 1.0f / (sh.lpart[ob][0][ra + 8] + sh.lpart[ob][1][ra + 8]);
-      W.wait(&B.o_full[ob], (is >> 1) & 1);
+      W.wait(&B.o_full, is & 1);
       tc_fence_after();
       float o[2 * D / 4];
 #pragma unroll
       for (int h = 0; h < D / 64; ++h) {
         uint32_t r[32];
-        ld_16x256b_x8(tmem + kColO + 128u * ob + 64u * h + lane_base, r);
+        ld_16x256b_x8(tmem + kColO + 64u * h + lane_base, r);
         tmem_wait_ld();
 #pragma unroll
         for (int jj = 0; jj < 32; ++jj) o[32 * h + jj] = __uint_as_float(r[jj]);
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&B.o_empty[ob]);
+      if (lane == 0) mbar_arrive(&B.o_empty);
       // All S steps of this item completed: its Q buffer takes item is + 2.
       load_q(is + 2);
       cp_async_wait<1>();               // this item's gates and coarse row (older group) landed
