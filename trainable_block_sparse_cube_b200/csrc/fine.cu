@@ -559,13 +559,17 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
         }
         // Optimistic pass with the current reference max. A thread's partial
         // row sum exceeds 2^8 whenever one of its scores exceeds the reference
-        // by more than 2^8 (and when the reference is still -inf), so only then
-        // are the exact row maxima needed.
+        // by more than 2^8, so only then are the exact row maxima needed. The
+        // first step of an item (reference still -inf) goes there directly.
         uint32_t pk[16];
-        float s0, s1;
-        if (masked) exp_pack<false>(r, scale, m0, m1, pk, s0, s1);
-        else exp_pack<true>(r, scale, m0, m1, pk, s0, s1);
-        if (pair_any(quarter, !(s0 <= 256.f) || !(s1 <= 256.f))) {
+        float s0 = 0.f, s1 = 0.f;
+        bool exact = true;
+        if (t > 0) {
+          if (masked) exp_pack<false>(r, scale, m0, m1, pk, s0, s1);
+          else exp_pack<true>(r, scale, m0, m1, pk, s0, s1);
+          exact = pair_any(quarter, !(s0 <= 256.f) || !(s1 <= 256.f));
+        }
+        if (exact) {
           float x0, x1;
           half_row_max(r, x0, x1);
           if ((lane & 3) == 0) {
