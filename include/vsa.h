@@ -80,7 +80,8 @@ typedef struct vsa_plan_s* vsa_plan_t;
 /* Byte offsets of the plan's workspace regions (for inspection by tests and
  * tools). All are relative to the workspace base passed to vsa_plan. */
 typedef struct {
-  size_t q_cube, k_cube, v_cube; /* [B*heads, C, 64, D] bf16, cube-major copies  */
+  size_t q_cube, k_cube, v_cube; /* [B*heads, C, 64, D] bf16, cube-major copies
+                                    (q's only with vsa_set_cube_major_copies)     */
   size_t q_pool, k_pool, v_pool; /* [B*heads, C, D] fp32 cube means               */
   size_t o_coarse;               /* [B*heads, C, D] fp32 coarse output            */
   size_t s_coarse;               /* [B*heads, C, C] fp32 coarse scores, overwritten
@@ -181,6 +182,15 @@ vsa_status vsa_set_wait_limit_ns(vsa_plan_t plan, uint64_t limit_ns);
  * signals, so that wait runs out after the plan's wait limit and the run
  * ends with VSA_ERR_TIMEOUT (reported by vsa_check) instead of hanging. */
 vsa_status vsa_set_debug_stall(vsa_plan_t plan, int on);
+
+/* Inspection switch for the gather step (raster -> cube-major reorder;
+ * "Faster Video Diffusion with Trainable Sparse Attention", "Approach": one
+ * cube of 4 x 4 x 4 tokens is one tile). Every run writes the cube-major
+ * copies of k and v (regions k_cube, v_cube), which the fine-attention kernel
+ * streams; it reads q straight from the raster tensor with 5-D TMA boxes, so
+ * q's copy is not needed. When `on` is nonzero, later runs of this plan also
+ * write q's copy into region q_cube (one extra write of q); off by default. */
+vsa_status vsa_set_cube_major_copies(vsa_plan_t plan, int on);
 
 /* Stage timing for benchmarks. When `on` is nonzero, later runs of this plan
  * record CUDA events (created here, once) on the run's stream around its three

@@ -92,6 +92,7 @@ def test_plan_argument_errors(lib):
     assert lib.vsa_check(None) == 1
     assert lib.vsa_set_wait_limit_ns(None, 10 ** 9) == 1
     assert lib.vsa_set_debug_stall(None, 1) == 1
+    assert lib.vsa_set_cube_major_copies(None, 1) == 1
     lib.vsa_plan_destroy(None)
 
 

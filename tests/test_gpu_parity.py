@@ -39,9 +39,10 @@ def _built():
     vsa.load()
 
 
-def _run(wl, inputs):
+def _run(wl, inputs, cube_copies=False):
     q, k, v, gc, gf = (t.cuda() for t in inputs)
     plan = vsa.Plan(wl.B, wl.heads, wl.T, wl.H, wl.W, wl.D, wl.topk, wl.top_p, wl.kmin, wl.kmax)
+    plan.set_cube_major_copies(cube_copies)
     out, idx, cnt = plan.run(q, k, v, gc, gf)
     plan.check()
     return plan, (q, k, v, gc, gf), out, idx, cnt
@@ -58,7 +59,7 @@ def _padded(lists, counts, kcap):
 def test_small_all_stages(wl):
     inputs = synth.make_inputs(wl)
     q, k, v, gc, gf = inputs
-    plan, dev_in, out, idx, cnt = _run(wl, inputs)
+    plan, dev_in, out, idx, cnt = _run(wl, inputs, cube_copies=True)
     perm = oracle.cube_perm(wl.T, wl.H, wl.W)
     BH = wl.B * wl.heads
     qc = plan.cube_major("q").cpu().view(wl.B, wl.heads, wl.C * 64, wl.D)

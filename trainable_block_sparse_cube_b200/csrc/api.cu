@@ -17,9 +17,12 @@ struct vsa_plan_s {
   int BH, N, C, kcap;
   char* ws;
   vsa_workspace_layout_t lay;
-  CUtensorMap tm_q, tm_k, tm_v;
+  CUtensorMap tm_q;         // raster map of q, encoded for the pointer tm_q_for
+  const void* tm_q_for;
+  CUtensorMap tm_k, tm_v;   // maps over the cube-major copies in the workspace
   CUtensorMap tm_out;       // output map, encoded for the output pointer tm_out_for
   const void* tm_out_for;
+  int cube_copies;          // also write q's cube-major copy (inspection)
   int num_sms;
   cudaStream_t last_stream;
   uint64_t wait_ns;
@@ -97,7 +100,8 @@ void make_layout(const vsa_config* c, vsa_workspace_layout_t* L) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-vsa_status encode_map(CUtensorMap* m, void* base, size_t rows, int D) {
+// 2-D map over a cube-major copy: rows of D bf16, 64 x 64 boxes, 128-byte swizzle.
+vsa_status encode_cube_map(CUtensorMap* m, void* base, size_t rows, int D) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return VSA_ERR_CUDA;
   cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
@@ -109,9 +113,10 @@ vsa_status encode_map(CUtensorMap* m, void* base, size_t rows, int D) {
   return r == CUDA_SUCCESS ? VSA_OK : VSA_ERR_CUDA;
 }
 
-// 5-D map over the raster output [BH][T][H][W][D] bf16: a box is one cube's
-// 4 x 4 x 4 tokens by 64 channels, stored from a 128-byte-swizzled tile.
-vsa_status encode_out_map(CUtensorMap* m, void* base, const vsa_config& c, int BH) {
+// 5-D map over a raster tensor [BH][T][H][W][D] bf16 (q or out): a box
+// is one cube's 4 x 4 x 4 tokens by 64 channels, laid out in shared memory as
+// 64 rows (in-cube slot order) of 128 bytes in the 128-byte swizzle.
+vsa_status encode_raster_map(CUtensorMap* m, const void* base, const vsa_config& c, int BH, bool load) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return VSA_ERR_CUDA;
   const cuuint64_t D = (cuuint64_t)c.D;
@@ -120,8 +125,10 @@ vsa_status encode_out_map(CUtensorMap* m, void* base, const vsa_config& c, int B
                            (cuuint64_t)c.T * c.H * c.W * D * 2};
   cuuint32_t box[5] = {64, 4, 4, 4, 1};
   cuuint32_t es[5] = {1, 1, 1, 1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   load ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? VSA_OK : VSA_ERR_CUDA;
 }
 
@@ -144,7 +151,7 @@ vsa_status run_common(vsa_plan_t P, const void* q, const void* k, const void* v,
   gp.src[0] = static_cast<const __nv_bfloat16*>(q);
   gp.src[1] = static_cast<const __nv_bfloat16*>(k);
   gp.src[2] = static_cast<const __nv_bfloat16*>(v);
-  gp.dst[0] = reinterpret_cast<__nv_bfloat16*>(ws + L.q_cube);
+  if (P->cube_copies) gp.dst[0] = reinterpret_cast<__nv_bfloat16*>(ws + L.q_cube);
   gp.dst[1] = reinterpret_cast<__nv_bfloat16*>(ws + L.k_cube);
   gp.dst[2] = reinterpret_cast<__nv_bfloat16*>(ws + L.v_cube);
   gp.pool[0] = reinterpret_cast<float*>(ws + L.q_pool);
@@ -169,10 +176,15 @@ vsa_status run_common(vsa_plan_t P, const void* q, const void* k, const void* v,
   if (vsa::launch_coarse(cp, st) != cudaSuccess) return VSA_ERR_CUDA;
 
   vsa::FineParams fp{};
+  if (P->tm_q_for != q) {
+    const vsa_status e = encode_raster_map(&P->tm_q, q, c, P->BH, true);
+    if (e != VSA_OK) return e;
+    P->tm_q_for = q;
+  }
   fp.tm_q = P->tm_q; fp.tm_k = P->tm_k; fp.tm_v = P->tm_v;
   if (out) {
     if (P->tm_out_for != out) {
-      const vsa_status e = encode_out_map(&P->tm_out, out, c, P->BH);
+      const vsa_status e = encode_raster_map(&P->tm_out, out, c, P->BH, false);
       if (e != VSA_OK) return e;
       P->tm_out_for = out;
     }
@@ -255,9 +267,8 @@ vsa_status vsa_plan(vsa_plan_t* out, const vsa_config* cfg, void* workspace, siz
   P->wait_ns = 1000000000ull;
   P->debug_stall = 0;
   const size_t rows = (size_t)P->BH * P->N;
-  vsa_status e = encode_map(&P->tm_q, P->ws + L.q_cube, rows, cfg->D);
-  if (e == VSA_OK) e = encode_map(&P->tm_k, P->ws + L.k_cube, rows, cfg->D);
-  if (e == VSA_OK) e = encode_map(&P->tm_v, P->ws + L.v_cube, rows, cfg->D);
+  vsa_status e = encode_cube_map(&P->tm_k, P->ws + L.k_cube, rows, cfg->D);
+  if (e == VSA_OK) e = encode_cube_map(&P->tm_v, P->ws + L.v_cube, rows, cfg->D);
   if (e == VSA_OK && cudaMemset(P->ws + L.err, 0, 16) != cudaSuccess) e = VSA_ERR_CUDA;
   if (e != VSA_OK) {
     delete P;
@@ -397,9 +408,8 @@ vsa_status vsa_forward_noalloc(const void* q, const void* k, const void* v, cons
   P.num_sms = sms;
   P.wait_ns = 1000000000ull;
   const size_t rows = (size_t)P.BH * P.N;
-  s = encode_map(&P.tm_q, P.ws + L.q_cube, rows, D);
-  if (s == VSA_OK) s = encode_map(&P.tm_k, P.ws + L.k_cube, rows, D);
-  if (s == VSA_OK) s = encode_map(&P.tm_v, P.ws + L.v_cube, rows, D);
+  s = encode_cube_map(&P.tm_k, P.ws + L.k_cube, rows, D);
+  if (s == VSA_OK) s = encode_cube_map(&P.tm_v, P.ws + L.v_cube, rows, D);
   if (s != VSA_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(P.ws + L.err, 0, 16, st) != cudaSuccess) return VSA_ERR_CUDA;
@@ -472,6 +482,12 @@ int vsa_kernels_per_run(void) { return 5; }
 vsa_status vsa_set_debug_stall(vsa_plan_t plan, int on) {
   if (!plan) return VSA_ERR_INVALID_ARG;
   plan->debug_stall = on ? 1 : 0;
+  return VSA_OK;
+}
+
+vsa_status vsa_set_cube_major_copies(vsa_plan_t plan, int on) {
+  if (!plan) return VSA_ERR_INVALID_ARG;
+  plan->cube_copies = on ? 1 : 0;
   return VSA_OK;
 }
 

@@ -13,6 +13,11 @@
 // item's selected KV cubes (128 keys):
 //   S[64 q x 128 keys] = Q . K_pair^T     tcgen05.mma M=64, N=128 (Q, K in smem)
 //   O[64 q x D]       += P . V_pair       tcgen05.mma M=64, N=D   (P in TMEM, V in smem)
+// Each query cube is read once, straight from the raster q: a 5-D TMA box of
+// 4 x 4 x 4 tokens by 64 channels lands as 64 rows in in-cube slot order. K
+// and V cubes, read about K times each from L2, come from the cube-major
+// copies (one contiguous 64 x D tile per cube), which load faster than the
+// strided raster boxes.
 //
 // Tensor memory holds three S/P buffers and the O accumulator: S of steps
 // j+1 and j+2 can run on the tensor core while the softmax works on step j,
@@ -420,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
         ca = ca < 0 || ca >= C ? 0 : ca;
         cb = cb < 0 || cb >= C ? 0 : cb;
       }
-      const int base_row = c.item / C * C;
+      const int bh = c.item / C;
       if (lane == 0) {
         const int slot = g % stages;
         if (g >= stages && !W.wait(&empty[slot], ((g / stages) - 1) & 1)) aborted = true;
@@ -429,8 +434,8 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
           uint8_t* dst = ring + slot * L::KV_BYTES;
 #pragma unroll
           for (int h = 0; h < L::NH; ++h) {
-            tma_load_2d(dst + h * 16384, tm, &full[slot], 64 * h, (base_row + ca) * 64);
-            tma_load_2d(dst + h * 16384 + 8192, tm, &full[slot], 64 * h, (base_row + cb) * 64);
+            tma_load_2d(dst + h * 16384, tm, &full[slot], 64 * h, (bh * C + ca) * 64);
+            tma_load_2d(dst + h * 16384 + 8192, tm, &full[slot], 64 * h, (bh * C + cb) * 64);
           }
         }
       }
@@ -641,10 +646,13 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
       const int b = is & 1;
       if (b == 0) ++qloads0; else ++qloads1;
       if (est == 0) {
+        const int bh = item / C, ci = item - bh * C;
+        const int ct = ci / (Hc * Wc), ch = (ci / Wc) % Hc, cw = ci % Wc;
         uint8_t* dst = tiles + L::OFF_Q + b * L::Q_BYTES;
         mbar_arrive_expect_tx(&B.q_full[b], L::Q_BYTES);
 #pragma unroll
-        for (int h = 0; h < L::NH; ++h) tma_load_2d(dst + h * 8192, &p.tm_q, &B.q_full[b], 64 * h, item * 64);
+        for (int h = 0; h < L::NH; ++h)
+          tma_load_5d(dst + h * 8192, &p.tm_q, &B.q_full[b], 64 * h, 4 * cw, 4 * ch, 4 * ct, bh);
       }
     };
     // Gates (16 runs of 4 raster tokens per gate array) and the coarse output

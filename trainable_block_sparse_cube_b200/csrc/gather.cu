@@ -2,10 +2,12 @@
 //
 // "Faster Video Diffusion with Trainable Sparse Attention", "Approach":
 // tokens are grouped into 4x4x4 cubes (one GPU tile per cube) and each cube
-// is mean-pooled to one coarse token. This kernel does both in one pass over
-// q, k and v: it copies each cube's 64 raster rows into one contiguous
-// 64 x D block of the cube-major workspace (bit copy) and writes the fp32
-// mean of the 64 rows.
+// is mean-pooled to one coarse token. This kernel reads each cube's 64 raster
+// rows of q, k and v once, writes the fp32 mean of the 64 rows and, for k and
+// v, copies the rows into one contiguous 64 x D block of the cube-major
+// workspace (bit copy), from which the fine kernel streams them. The fine
+// kernel reads q straight from its raster layout, so q's copy is written
+// only when a plan asks for it for inspection.
 //
 // One warp per (tensor, head, cube). A raster row of D bf16 is D*2 bytes; a
 // lane moves 16 bytes, so D/8 lanes cover a row and a warp covers 32/(D/8)
@@ -27,7 +29,8 @@ __global__ void __launch_bounds__(256) gather_pool_kernel(const GatherParams p) 
   if (c >= p.C) return;
   const int sub = lane / LPR, chunk = lane % LPR;
   const __nv_bfloat16* src = p.src[tensor] + (size_t)bh * p.N * D + chunk * 8;
-  __nv_bfloat16* dst = p.dst[tensor] + ((size_t)bh * p.C + c) * kCube * D + chunk * 8;
+  const bool copy = p.dst[tensor] != nullptr;  // uniform over the grid's z slice
+  __nv_bfloat16* dst = copy ? p.dst[tensor] + ((size_t)bh * p.C + c) * kCube * D + chunk * 8 : nullptr;
 
   float acc[8];
 #pragma unroll
@@ -46,7 +49,7 @@ __global__ void __launch_bounds__(256) gather_pool_kernel(const GatherParams p) 
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int r = (s0 + u) * RPS + sub;
-      *reinterpret_cast<int4*>(dst + (size_t)r * D) = v[u];
+      if (copy) *reinterpret_cast<int4*>(dst + (size_t)r * D) = v[u];
       const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {

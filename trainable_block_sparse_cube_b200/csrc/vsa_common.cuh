@@ -23,7 +23,7 @@ __host__ __device__ __forceinline__ int cube_token(int c, int r, int H, int W) {
 
 struct GatherParams {
   const __nv_bfloat16* src[3];  // q, k, v raster [BH, N, D]
-  __nv_bfloat16* dst[3];        // cube-major [BH, C, 64, D]
+  __nv_bfloat16* dst[3];        // cube-major [BH, C, 64, D]; null: pool only for that tensor
   float* pool[3];               // [BH, C, D] cube means
   int BH, C, H, W, N;
 };
@@ -46,8 +46,11 @@ struct CoarseParams {
 };
 
 struct FineParams {
-  CUtensorMap tm_q, tm_k, tm_v;  // 2-D maps over the cube-major copies, rows of D bf16
-  CUtensorMap tm_out;            // 5-D map over out [BH][T][H][W][D], 64-column boxes of one cube, 128 B swizzle
+  // tm_q, tm_out: 5-D maps over the raster q and out [BH][T][H][W][D] bf16; a
+  // box is one cube's 4 x 4 x 4 tokens by 64 channels, in the 128-byte swizzle.
+  // tm_k, tm_v: 2-D maps over the cube-major copies (rows of D bf16, 64 x 64 boxes).
+  CUtensorMap tm_q, tm_k, tm_v;
+  CUtensorMap tm_out;
   const int32_t* idx;            // [BH, C, kcap]
   const int32_t* cnt;            // [BH, C] or null (then every row has kcap ids)
   const float* oc;               // [BH, C, D]

@@ -21,7 +21,7 @@ STATUS = {0: "VSA_OK", 1: "VSA_ERR_INVALID_ARG", 2: "VSA_ERR_SHAPE", 3: "VSA_ERR
 EXPORTED = ["vsa_workspace_bytes", "vsa_workspace_layout", "vsa_plan", "vsa_run", "vsa_run_fixed_idx",
             "vsa_forward", "vsa_check", "vsa_plan_destroy", "vsa_status_string", "vsa_set_wait_limit_ns",
             "vsa_set_debug_stall", "vsa_set_stage_timing", "vsa_stage_times", "vsa_kernels_per_run",
-            "vsa_forward_noalloc"]
+            "vsa_forward_noalloc", "vsa_set_cube_major_copies"]
 
 
 class VSAError(RuntimeError):
@@ -75,6 +75,8 @@ def load():
     L.vsa_set_wait_limit_ns.restype = i32
     L.vsa_set_debug_stall.argtypes = [vp, i32]
     L.vsa_set_debug_stall.restype = i32
+    L.vsa_set_cube_major_copies.argtypes = [vp, i32]
+    L.vsa_set_cube_major_copies.restype = i32
     L.vsa_set_stage_timing.argtypes = [vp, i32]
     L.vsa_set_stage_timing.restype = i32
     L.vsa_stage_times.argtypes = [vp, ctypes.POINTER(ctypes.c_float)]
@@ -195,6 +197,10 @@ class Plan:
 
     def set_debug_stall(self, on: bool):
         _check(load().vsa_set_debug_stall(self._h, 1 if on else 0), "vsa_set_debug_stall")
+
+    def set_cube_major_copies(self, on: bool):
+        """Also write the cube-major copy of q into the workspace (k and v are always copied)."""
+        _check(load().vsa_set_cube_major_copies(self._h, 1 if on else 0), "vsa_set_cube_major_copies")
 
     def set_stage_timing(self, on: bool):
         _check(load().vsa_set_stage_timing(self._h, 1 if on else 0), "vsa_set_stage_timing")
