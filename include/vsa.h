@@ -86,6 +86,10 @@ typedef struct {
   size_t o_coarse;               /* [B*heads, C, D] fp32 coarse output            */
   size_t s_coarse;               /* [B*heads, C, C] fp32 coarse scores, overwritten
                                     by the coarse softmax probabilities           */
+  size_t o_part;                 /* [4, B*heads, C, D] fp32 partial products of the
+                                    coarse output (K split over several CTAs)     */
+  size_t tile_cnt;               /* [B*heads, ceil(C/64)] int32 arrival counts of
+                                    those partials; zero between runs             */
   size_t cnt;                    /* [B*heads, C] int32 counts used by the fine step */
   size_t err;                    /* int32 device error word                        */
   size_t total;                  /* == vsa_workspace_bytes                          */

@@ -54,6 +54,9 @@ EncodeTiledFn get_encode_fn() {
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 constexpr int kMaxC = 4096;
+constexpr int kOutSplitsMax = 4;
+// K splits of the coarse output GEMM: enough CTAs to fill the GPU at large C.
+inline int out_splits(int C) { return C >= 512 ? 4 : (C >= 256 ? 2 : 1); }
 constexpr int kMaxTopPKmax = 1024;
 
 vsa_status validate(const vsa_config* c) {
@@ -93,6 +96,8 @@ void make_layout(const vsa_config* c, vsa_workspace_layout_t* L) {
   L->v_pool = take(BH * C * D * 4);
   L->o_coarse = take(BH * C * D * 4);
   L->s_coarse = take(BH * C * C * 4);
+  L->o_part = take(kOutSplitsMax * BH * C * D * 4);
+  L->tile_cnt = take(BH * ((C + 63) / 64) * 4);
   L->cnt = take(BH * C * 4);
   L->err = take(16);
   L->total = off;
@@ -167,6 +172,9 @@ vsa_status run_common(vsa_plan_t P, const void* q, const void* k, const void* v,
   cp.s = reinterpret_cast<float*>(ws + L.s_coarse);
   cp.oc = reinterpret_cast<float*>(ws + L.o_coarse);
   cp.oc_copy = out_coarse;
+  cp.opart = reinterpret_cast<float*>(ws + L.o_part);
+  cp.tile_cnt = reinterpret_cast<int*>(ws + L.tile_cnt);
+  cp.splits = out_splits(P->C);
   cp.idx = idx_out;
   cp.cnt = reinterpret_cast<int32_t*>(ws + L.cnt);
   cp.BH = P->BH; cp.C = P->C; cp.D = c.D; cp.kcap = P->kcap;
@@ -270,6 +278,7 @@ vsa_status vsa_plan(vsa_plan_t* out, const vsa_config* cfg, void* workspace, siz
   vsa_status e = encode_cube_map(&P->tm_k, P->ws + L.k_cube, rows, cfg->D);
   if (e == VSA_OK) e = encode_cube_map(&P->tm_v, P->ws + L.v_cube, rows, cfg->D);
   if (e == VSA_OK && cudaMemset(P->ws + L.err, 0, 16) != cudaSuccess) e = VSA_ERR_CUDA;
+  if (e == VSA_OK && cudaMemset(P->ws + L.tile_cnt, 0, L.cnt - L.tile_cnt) != cudaSuccess) e = VSA_ERR_CUDA;
   if (e != VSA_OK) {
     delete P;
     return e;
@@ -413,6 +422,7 @@ vsa_status vsa_forward_noalloc(const void* q, const void* k, const void* v, cons
   if (s != VSA_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(P.ws + L.err, 0, 16, st) != cudaSuccess) return VSA_ERR_CUDA;
+  if (cudaMemsetAsync(P.ws + L.tile_cnt, 0, L.cnt - L.tile_cnt, st) != cudaSuccess) return VSA_ERR_CUDA;
   return run_common(&P, q, k, v, gate_c, gate_f, true, nullptr, nullptr, idx, nullptr, out, nullptr, nullptr,
                     stream);
 }

@@ -35,6 +35,9 @@ struct CoarseParams {
   float* s;            // [BH, C, C] scores, then probabilities
   float* oc;           // [BH, C, D]
   float* oc_copy;      // optional second destination of oc (may be null)
+  float* opart;        // [splits, BH, C, D] partial products of the output GEMM
+  int* tile_cnt;       // [BH, ceil(C/64)] arrival counts (zero between runs)
+  int splits;          // K splits of the output GEMM (1: no partials)
   int32_t* idx;        // [BH, C, kcap]
   int32_t* cnt;        // [BH, C]
   int BH, C, D, kcap;

@@ -38,7 +38,8 @@ class Config(ctypes.Structure):
 
 class WorkspaceLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in ("q_cube", "k_cube", "v_cube", "q_pool", "k_pool", "v_pool",
-                                               "o_coarse", "s_coarse", "cnt", "err", "total")]
+                                               "o_coarse", "s_coarse", "o_part", "tile_cnt", "cnt", "err",
+                                               "total")]
 
 
 _lib = None
