@@ -263,8 +263,9 @@ __device__ __forceinline__ uint32_t kth_largest(const uint32_t (&key)[PER], int 
   return T;
 }
 
-template <int PER>
-__global__ void __launch_bounds__(256) coarse_select_kernel(const CoarseParams p) {
+// TOPK: fixed top-K (no top-p scratch, fewer registers, more warps per SM).
+template <int PER, bool TOPK>
+__global__ void __launch_bounds__(256, TOPK ? 3 : 1) coarse_select_kernel(const CoarseParams p) {
   extern __shared__ __align__(16) uint8_t dyn[];
   __shared__ uint32_t cand_all[8][kCandCap];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -302,7 +303,7 @@ __global__ void __launch_bounds__(256) coarse_select_kernel(const CoarseParams p
 
     int32_t* irow = p.idx + (size_t)row * p.kcap;
     int n_out;
-    if (p.topk > 0) {
+    if (TOPK) {
       int pos = 0, eq_seen = 0;
 #pragma unroll
       for (int u = 0; u < PER; ++u) {
@@ -468,13 +469,17 @@ __global__ void __launch_bounds__(kGThreads) coarse_output_kernel(const CoarsePa
 template <int PER>
 cudaError_t launch_select(const CoarseParams& p, cudaStream_t st) {
   const int rows = p.BH * p.C;
-  const size_t smem = (p.do_select && p.topk == 0) ? (size_t)8 * p.kmax * 16 : 0;
+  if (!p.do_select || p.topk > 0) {
+    coarse_select_kernel<PER, true><<<(rows + 7) / 8, 256, 0, st>>>(p);
+    return cudaGetLastError();
+  }
+  const size_t smem = (size_t)8 * p.kmax * 16;
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(coarse_select_kernel<PER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(coarse_select_kernel<PER, false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  coarse_select_kernel<PER><<<(rows + 7) / 8, 256, smem, st>>>(p);
+  coarse_select_kernel<PER, false><<<(rows + 7) / 8, 256, smem, st>>>(p);
   return cudaGetLastError();
 }
 
