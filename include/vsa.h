@@ -84,12 +84,12 @@ typedef struct {
                                     (q's only with vsa_set_cube_major_copies)     */
   size_t q_pool, k_pool, v_pool; /* [B*heads, C, D] fp32 cube means               */
   size_t o_coarse;               /* [B*heads, C, D] fp32 coarse output            */
-  size_t s_coarse;               /* [B*heads, C, C] fp32 coarse scores, overwritten
-                                    by the coarse softmax probabilities           */
-  size_t o_part;                 /* [4, B*heads, C, D] fp32 partial products of the
-                                    coarse output (K split over several CTAs)     */
-  size_t tile_cnt;               /* [B*heads, ceil(C/64)] int32 arrival counts of
-                                    those partials; zero between runs             */
+  size_t s_coarse;               /* [B*heads, C, C] fp32 coarse scores             */
+  size_t pool_split;             /* [3 (q, k, v), 3, B*heads, C, D] bf16: each cube
+                                    mean as three bf16 terms hi + mid + lo        */
+  size_t p_split;                /* [3, B*heads, C, Cp] bf16: the coarse softmax
+                                    probabilities as three bf16 terms, Cp = C
+                                    rounded up to a multiple of 8 (zero padded)   */
   size_t cnt;                    /* [B*heads, C] int32 counts used by the fine step */
   size_t err;                    /* int32 device error word                        */
   size_t total;                  /* == vsa_workspace_bytes                          */

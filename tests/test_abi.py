@@ -74,12 +74,12 @@ def test_layout_sizes(lib):
     BH, N, C, D = 6, 8 * 12 * 16, 8 * 12 * 16 // 64, 128
     assert lay.k_cube - lay.q_cube >= BH * N * D * 2
     assert lay.q_pool - lay.v_cube >= BH * N * D * 2
-    assert lay.o_part - lay.s_coarse >= BH * C * C * 4
+    assert lay.pool_split - lay.s_coarse >= BH * C * C * 4
     assert lay.total == lib.vsa_workspace_bytes(ctypes.byref(c))
-    assert lay.tile_cnt - lay.o_part >= 4 * BH * C * D * 4
-    assert lay.cnt - lay.tile_cnt >= BH * ((C + 63) // 64) * 4
+    assert lay.p_split - lay.pool_split >= 9 * BH * C * D * 2
+    assert lay.cnt - lay.p_split >= 3 * BH * C * ((C + 7) // 8 * 8) * 2
     offs = [lay.q_cube, lay.k_cube, lay.v_cube, lay.q_pool, lay.k_pool, lay.v_pool, lay.o_coarse, lay.s_coarse,
-            lay.o_part, lay.tile_cnt, lay.cnt, lay.err]
+            lay.pool_split, lay.p_split, lay.cnt, lay.err]
     assert offs == sorted(offs) and all(o % 1024 == 0 for o in offs)
 
 

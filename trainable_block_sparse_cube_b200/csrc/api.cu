@@ -20,6 +20,7 @@ struct vsa_plan_s {
   CUtensorMap tm_q;         // raster map of q, encoded for the pointer tm_q_for
   const void* tm_q_for;
   CUtensorMap tm_k, tm_v;   // maps over the cube-major copies in the workspace
+  CUtensorMap tm_qs, tm_ks, tm_vs, tm_ps;  // maps over the coarse operands' bf16 terms
   CUtensorMap tm_out;       // output map, encoded for the output pointer tm_out_for
   const void* tm_out_for;
   int cube_copies;          // also write q's cube-major copy (inspection)
@@ -54,9 +55,8 @@ EncodeTiledFn get_encode_fn() {
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 constexpr int kMaxC = 4096;
-constexpr int kOutSplitsMax = 4;
-// K splits of the coarse output GEMM: enough CTAs to fill the GPU at large C.
-inline int out_splits(int C) { return C >= 512 ? 4 : (C >= 256 ? 2 : 1); }
+// Row pitch of the coarse probabilities' bf16 terms: C rounded up to 8 (16 bytes).
+inline size_t coarse_pitch(size_t C) { return (C + 7) / 8 * 8; }
 constexpr int kMaxTopPKmax = 1024;
 
 vsa_status validate(const vsa_config* c) {
@@ -96,8 +96,8 @@ void make_layout(const vsa_config* c, vsa_workspace_layout_t* L) {
   L->v_pool = take(BH * C * D * 4);
   L->o_coarse = take(BH * C * D * 4);
   L->s_coarse = take(BH * C * C * 4);
-  L->o_part = take(kOutSplitsMax * BH * C * D * 4);
-  L->tile_cnt = take(BH * ((C + 63) / 64) * 4);
+  L->pool_split = take(9 * BH * C * D * 2);
+  L->p_split = take(3 * BH * C * coarse_pitch(C) * 2);
   L->cnt = take(BH * C * 4);
   L->err = take(16);
   L->total = off;
@@ -116,6 +116,34 @@ vsa_status encode_cube_map(CUtensorMap* m, void* base, size_t rows, int D) {
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? VSA_OK : VSA_ERR_CUDA;
+}
+
+// 3-D map over [planes][rows][cols] bf16 (row pitch `pitch` elements), boxes of
+// box_rows x 64 columns in the 128-byte swizzle.
+vsa_status encode_planes_map(CUtensorMap* m, void* base, size_t cols, size_t pitch, size_t rows, size_t planes,
+                             int box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return VSA_ERR_CUDA;
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)planes};
+  cuuint64_t strides[2] = {(cuuint64_t)pitch * 2, (cuuint64_t)pitch * rows * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? VSA_OK : VSA_ERR_CUDA;
+}
+
+// Maps over the bf16 terms of the pooled q, k, v ([3 * BH][C][D] each) and of
+// the coarse probabilities ([3 * BH][C][Cp]).
+vsa_status encode_coarse_maps(vsa_plan_s* P) {
+  const size_t BH = P->BH, C = P->C, D = P->cfg.D, Cp = coarse_pitch(C);
+  char* base = P->ws + P->lay.pool_split;
+  const size_t tbytes = 3 * BH * C * D * 2;
+  vsa_status e = encode_planes_map(&P->tm_qs, base, D, D, C, 3 * BH, 128);
+  if (e == VSA_OK) e = encode_planes_map(&P->tm_ks, base + tbytes, D, D, C, 3 * BH, 128);
+  if (e == VSA_OK) e = encode_planes_map(&P->tm_vs, base + 2 * tbytes, D, D, C, 3 * BH, 64);
+  if (e == VSA_OK) e = encode_planes_map(&P->tm_ps, P->ws + P->lay.p_split, Cp, Cp, C, 3 * BH, 128);
+  return e;
 }
 
 // 5-D map over a raster tensor [BH][T][H][W][D] bf16 (q or out): a box
@@ -162,19 +190,22 @@ vsa_status run_common(vsa_plan_t P, const void* q, const void* k, const void* v,
   gp.pool[0] = reinterpret_cast<float*>(ws + L.q_pool);
   gp.pool[1] = reinterpret_cast<float*>(ws + L.k_pool);
   gp.pool[2] = reinterpret_cast<float*>(ws + L.v_pool);
+  for (int t = 0; t < 3; ++t)
+    gp.split[t] = reinterpret_cast<__nv_bfloat16*>(ws + L.pool_split + (size_t)t * 3 * P->BH * P->C * c.D * 2);
   gp.BH = P->BH; gp.C = P->C; gp.H = c.H; gp.W = c.W; gp.N = P->N;
   if (P->timing && cudaEventRecord(P->ev[0], st) != cudaSuccess) return VSA_ERR_CUDA;
   if (vsa::launch_gather(gp, c.D, st) != cudaSuccess) return VSA_ERR_CUDA;
   if (P->timing && cudaEventRecord(P->ev[1], st) != cudaSuccess) return VSA_ERR_CUDA;
 
   vsa::CoarseParams cp{};
-  cp.qpool = gp.pool[0]; cp.kpool = gp.pool[1]; cp.vpool = gp.pool[2];
+  cp.tm_qs = P->tm_qs; cp.tm_ks = P->tm_ks; cp.tm_vs = P->tm_vs; cp.tm_ps = P->tm_ps;
+  cp.psplit = reinterpret_cast<__nv_bfloat16*>(ws + L.p_split);
+  cp.Cp = (int)coarse_pitch(P->C);
+  cp.err = reinterpret_cast<int*>(ws + L.err);
+  cp.wait_ns = P->wait_ns;
   cp.s = reinterpret_cast<float*>(ws + L.s_coarse);
   cp.oc = reinterpret_cast<float*>(ws + L.o_coarse);
   cp.oc_copy = out_coarse;
-  cp.opart = reinterpret_cast<float*>(ws + L.o_part);
-  cp.tile_cnt = reinterpret_cast<int*>(ws + L.tile_cnt);
-  cp.splits = out_splits(P->C);
   cp.idx = idx_out;
   cp.cnt = reinterpret_cast<int32_t*>(ws + L.cnt);
   cp.BH = P->BH; cp.C = P->C; cp.D = c.D; cp.kcap = P->kcap;
@@ -277,8 +308,8 @@ vsa_status vsa_plan(vsa_plan_t* out, const vsa_config* cfg, void* workspace, siz
   const size_t rows = (size_t)P->BH * P->N;
   vsa_status e = encode_cube_map(&P->tm_k, P->ws + L.k_cube, rows, cfg->D);
   if (e == VSA_OK) e = encode_cube_map(&P->tm_v, P->ws + L.v_cube, rows, cfg->D);
+  if (e == VSA_OK) e = encode_coarse_maps(P);
   if (e == VSA_OK && cudaMemset(P->ws + L.err, 0, 16) != cudaSuccess) e = VSA_ERR_CUDA;
-  if (e == VSA_OK && cudaMemset(P->ws + L.tile_cnt, 0, L.cnt - L.tile_cnt) != cudaSuccess) e = VSA_ERR_CUDA;
   if (e != VSA_OK) {
     delete P;
     return e;
@@ -419,10 +450,10 @@ vsa_status vsa_forward_noalloc(const void* q, const void* k, const void* v, cons
   const size_t rows = (size_t)P.BH * P.N;
   s = encode_cube_map(&P.tm_k, P.ws + L.k_cube, rows, D);
   if (s == VSA_OK) s = encode_cube_map(&P.tm_v, P.ws + L.v_cube, rows, D);
+  if (s == VSA_OK) s = encode_coarse_maps(&P);
   if (s != VSA_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(P.ws + L.err, 0, 16, st) != cudaSuccess) return VSA_ERR_CUDA;
-  if (cudaMemsetAsync(P.ws + L.tile_cnt, 0, L.cnt - L.tile_cnt, st) != cudaSuccess) return VSA_ERR_CUDA;
   return run_common(&P, q, k, v, gate_c, gate_f, true, nullptr, nullptr, idx, nullptr, out, nullptr, nullptr,
                     stream);
 }

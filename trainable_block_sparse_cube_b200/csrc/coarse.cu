@@ -8,16 +8,21 @@
 // may keep a variable number of key-value blocks; here that is the top-p
 // rule documented in include/vsa.h.
 //
-// Three launches per call, all in fp32 on the CUDA cores (the scores decide
-// integer selections, so they are kept in fp32 rather than bf16):
-//   1. scores   s = qbar kbar^T / sqrt(D)       [BH, C, C]   (tiled SGEMM, 64 x 128 tiles)
+// Three launches per call. The scores decide integer selections, so both
+// products keep fp32 accuracy; they run on the tensor cores by writing every
+// fp32 operand x as three bf16 terms x = hi + mid + lo (8 significant bits
+// each, |x - hi - mid - lo| <= 2^-25 |x|) and summing the six products
+// hi.hi, hi.mid, mid.hi, mid.mid, hi.lo, lo.hi in fp32 tensor memory; the
+// dropped ones are below 2^-24 relative.
+//   1. scores   s = qbar kbar^T / sqrt(D)       [BH, C, C]   (tcgen05, 128 x 128 tiles)
 //   2. select   row max / sum, exact K-th largest score by a 32-step radix
 //               search on order-preserving integer keys (one warp per row,
 //               keys in registers), ascending index lists with ties to the
 //               lower id; top-p ranks the kmax best candidates and cuts at
-//               the first prefix whose mass reaches p. Writes P over s.
-//   3. output   Oc = P vbar                     [BH, C, D]   (tiled SGEMM, K split over
-//               several CTAs per tile, partials added in a fixed order)
+//               the first prefix whose mass reaches p. Writes P as three
+//               bf16 terms.
+//   3. output   Oc = P vbar                     [BH, C, D]   (tcgen05, 128 x D tiles)
+#include "sm100_ptx.cuh"
 #include "vsa_common.cuh"
 
 namespace vsa {
@@ -40,146 +45,6 @@ __device__ __forceinline__ float key_value(uint32_t k) {
 }
 
 constexpr float kLog2e = 1.4426950408889634f;
-
-// ------------------------------------------------------------ fp32 GEMM tile
-// One CTA computes a 64 x 128 tile of A . B over a range of K with 128
-// threads, 8 x 8 outputs per thread (rows {4ty + i, 32 + 4ty + i}, columns
-// {4tx + j, 64 + 4tx + j}), in steps of 16 along K staged through shared
-// memory twice over so the global loads of step k+1 overlap the FMAs of
-// step k.
-//   A: row-major [M x K] (element (m, k) at A[m * lda + k]).
-//   B: B_KMAJOR ? row-major [N x K] (element (n, k) at B[n * ldb + k])
-//               : row-major [K x N] (element (k, n) at B[k * ldb + n]).
-constexpr int kGM = 64, kGN = 128, kGK = 16, kGThreads = 128;
-
-struct GemmSmem {
-  float a[2][kGK][kGM + 4];  // [k][m]
-  float b[2][kGK][kGN + 4];  // [k][n]
-};
-
-template <bool B_KMAJOR>
-struct GemmTile {
-  const float* A;
-  const float* B;
-  int lda, ldb, M, N;
-  bool a_vec;  // A rows 16-byte aligned: float4 loads
-  float ra[8], rb[16];
-
-  __device__ __forceinline__ void load(int m0, int n0, int k0, int k_end) {
-    const int tid = threadIdx.x;
-    {  // A: row m0 + tid / 2, k0 + 8 (tid % 2) .. + 7
-      const int m = m0 + (tid >> 1), kb = k0 + (tid & 1) * 8;
-      const float* src = A + (size_t)m * lda + kb;
-      if (a_vec && m < M && kb + 8 <= k_end) {
-        const float4 x = *reinterpret_cast<const float4*>(src);
-        const float4 y = *reinterpret_cast<const float4*>(src + 4);
-        ra[0] = x.x; ra[1] = x.y; ra[2] = x.z; ra[3] = x.w;
-        ra[4] = y.x; ra[5] = y.y; ra[6] = y.z; ra[7] = y.w;
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) ra[e] = (m < M && kb + e < k_end) ? src[e] : 0.f;
-      }
-    }
-    if (B_KMAJOR) {  // B: row n0 + tid, k0 .. k0 + 15
-      const int n = n0 + tid;
-      const float* src = B + (size_t)n * ldb + k0;
-      if (n < N && k0 + 16 <= k_end) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float4 x = *reinterpret_cast<const float4*>(src + 4 * q);
-          rb[4 * q] = x.x; rb[4 * q + 1] = x.y; rb[4 * q + 2] = x.z; rb[4 * q + 3] = x.w;
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 16; ++e) rb[e] = (n < N && k0 + e < k_end) ? src[e] : 0.f;
-      }
-    } else {  // B: row k0 + tid / 8, columns n0 + 16 (tid % 8) .. + 15
-      const int k = k0 + (tid >> 3), nb = n0 + (tid & 7) * 16;
-      const float* src = B + (size_t)k * ldb + nb;
-      if (k < k_end && nb + 16 <= N) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float4 x = *reinterpret_cast<const float4*>(src + 4 * q);
-          rb[4 * q] = x.x; rb[4 * q + 1] = x.y; rb[4 * q + 2] = x.z; rb[4 * q + 3] = x.w;
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 16; ++e) rb[e] = (k < k_end && nb + e < N) ? src[e] : 0.f;
-      }
-    }
-  }
-
-  __device__ __forceinline__ void store(GemmSmem& sm, int buf) const {
-    const int tid = threadIdx.x;
-    const int m = tid >> 1, kb = (tid & 1) * 8;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) sm.a[buf][kb + e][m] = ra[e];
-    if (B_KMAJOR) {
-#pragma unroll
-      for (int e = 0; e < 16; ++e) sm.b[buf][e][tid] = rb[e];
-    } else {
-      const int k = tid >> 3, nb = (tid & 7) * 16;
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        *reinterpret_cast<float4*>(&sm.b[buf][k][nb + 4 * q]) =
-            make_float4(rb[4 * q], rb[4 * q + 1], rb[4 * q + 2], rb[4 * q + 3]);
-    }
-  }
-
-  // acc += A[m0.., k_begin..k_end) . B[.., n0..]
-  __device__ __forceinline__ void run(GemmSmem& sm, int m0, int n0, int k_begin, int k_end, float (&acc)[8][8]) {
-    const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
-    int buf = 0;
-    load(m0, n0, k_begin, k_end);
-    store(sm, 0);
-    __syncthreads();
-    for (int k0 = k_begin; k0 < k_end; k0 += kGK) {
-      const bool more = k0 + kGK < k_end;
-      if (more) load(m0, n0, k0 + kGK, k_end);
-#pragma unroll
-      for (int kk = 0; kk < kGK; ++kk) {
-        const float4 a0 = *reinterpret_cast<const float4*>(&sm.a[buf][kk][4 * ty]);
-        const float4 a1 = *reinterpret_cast<const float4*>(&sm.a[buf][kk][32 + 4 * ty]);
-        const float4 b0 = *reinterpret_cast<const float4*>(&sm.b[buf][kk][4 * tx]);
-        const float4 b1 = *reinterpret_cast<const float4*>(&sm.b[buf][kk][64 + 4 * tx]);
-        const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-        const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-#pragma unroll
-          for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-      }
-      if (more) store(sm, buf ^ 1);
-      __syncthreads();
-      buf ^= 1;
-    }
-  }
-};
-
-// Row and column of accumulator (i, j) of this thread within the 64 x 128 tile.
-__device__ __forceinline__ int tile_row(int i) { return (i < 4 ? 0 : 32) + 4 * (threadIdx.x >> 4) + (i & 3); }
-__device__ __forceinline__ int tile_col(int j) { return (j < 4 ? 0 : 64) + 4 * (threadIdx.x & 15) + (j & 3); }
-
-// ------------------------------------------------------------ 1. scores
-__global__ void __launch_bounds__(kGThreads) coarse_scores_kernel(const CoarseParams p) {
-  __shared__ __align__(16) GemmSmem sm;
-  const int C = p.C, D = p.D;
-  const int bh = blockIdx.z, m0 = blockIdx.y * kGM, n0 = blockIdx.x * kGN;
-  GemmTile<true> g{p.qpool + (size_t)bh * C * D, p.kpool + (size_t)bh * C * D, D, D, C, C, true};
-  float acc[8][8] = {};
-  g.run(sm, m0, n0, 0, D, acc);
-  float* S = p.s + (size_t)bh * C * C;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int r = m0 + tile_row(i);
-    if (r >= C) continue;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int c = n0 + tile_col(j);
-      if (c < C) S[(size_t)r * C + c] = acc[i][j] * p.scale;
-    }
-  }
-}
 
 // ------------------------------------------------------------ 2. select
 __device__ __forceinline__ float warp_max(float v) {
@@ -392,78 +257,182 @@ __global__ void __launch_bounds__(256, TOPK ? 3 : 1) coarse_select_kernel(const 
     for (int c = n_out + lane; c < p.kcap; c += 32) irow[c] = -1;
     if (lane == 0) p.cnt[row] = n_out;
   }
-  // Probabilities over the scores (read back by the output SGEMM).
+  // Probabilities over the scores as three bf16 terms (zero in the padding
+  // columns C .. Cp-1), the A operand of the output product.
   const float inv_l = 1.0f / l;
+  const size_t plane = (size_t)p.BH * C * p.Cp;
+  __nv_bfloat16* prow = p.psplit + (size_t)row * p.Cp;
 #pragma unroll
   for (int u = 0; u < PER; ++u) {
     const int j = lane + 32 * u;
-    if (j < C) srow[j] = fast_exp2(fmaf(key_value(key[u]), kLog2e, -mb)) * inv_l;
+    if (j < p.Cp) {
+      const float x = j < C ? fast_exp2(fmaf(key_value(key[u]), kLog2e, -mb)) * inv_l : 0.f;
+      const __nv_bfloat16 h = __float2bfloat16_rn(x);
+      const float r1 = x - __bfloat162float(h);
+      const __nv_bfloat16 m = __float2bfloat16_rn(r1);
+      prow[j] = h;
+      prow[plane + j] = m;
+      prow[2 * plane + j] = __float2bfloat16_rn(r1 - __bfloat162float(m));
+    }
   }
 }
 
-// ------------------------------------------------------------ 3. output
-// Oc = P . vbar with K (the C key cubes) split into p.splits ranges: each CTA
-// writes the partial product of its range, and the last CTA of a tile (an
-// atomic arrival count) adds the partials in split order, so the sum is the
-// same on every run.
-__global__ void __launch_bounds__(kGThreads) coarse_output_kernel(const CoarseParams p) {
-  __shared__ __align__(16) GemmSmem sm;
-  __shared__ int last;
-  const int C = p.C, D = p.D, S = p.splits;
-  const int bh = blockIdx.z, split = blockIdx.y, mt = blockIdx.x, m0 = mt * kGM;
-  const int kper = (((C + S - 1) / S) + kGK - 1) / kGK * kGK;
-  const int kb = split * kper, ke = min(C, kb + kper);
-  GemmTile<false> g{p.s + (size_t)bh * C * C, p.vpool + (size_t)bh * C * D, C, D, C, D, (C & 3) == 0};
-  float acc[8][8] = {};
-  if (kb < ke) g.run(sm, m0, 0, kb, ke, acc);
-  float* dst = S == 1 ? p.oc + (size_t)bh * C * D : p.opart + ((size_t)split * p.BH + bh) * C * D;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int r = m0 + tile_row(i);
-    if (r >= C) continue;
-#pragma unroll
-    for (int jb = 0; jb < 8; jb += 4) {
-      const int c = tile_col(jb);
-      if (c < D) *reinterpret_cast<float4*>(dst + (size_t)r * D + c) =
-                     make_float4(acc[i][jb], acc[i][jb + 1], acc[i][jb + 2], acc[i][jb + 3]);
+// ------------------------------------------------------------ 1 / 3. three-term bf16 GEMM
+// One CTA per 128-row tile: warp 0 issues the TMA loads (all three terms of A
+// and B for 64 columns of K per stage, two stages), warp 1 the 6 x 4 MMAs of
+// a stage (M=128, K=16 each), and all four warps read the fp32 accumulator
+// out of tensor memory.
+//   KIND 0 (scores): A = qbar terms [C x D], B = kbar terms [C x D] (both
+//          K-major), N tile 128 key cubes, K = D; out = S * scale.
+//   KIND 1 (output): A = P terms [C x Cp] (K-major), B = vbar terms [C x D]
+//          (N-major), N = D, K = Cp; out = Oc (and the optional copy).
+// Every wait is bounded; a wait that gives up records kErrTimeout.
+template <int KIND, int D>
+struct TcShape {
+  static constexpr int NT = KIND == 0 ? 128 : D;    // accumulator columns
+  static constexpr int A_BYTES = 128 * 64 * 2;      // one term, 128 rows x 64 K
+  static constexpr int B_BYTES = NT * 64 * 2;       // one term
+  static constexpr int STAGE = 3 * (A_BYTES + B_BYTES);
+  static constexpr int SMEM = 2 * STAGE + 1024;
+};
+
+template <int KIND, int D>
+__global__ void __launch_bounds__(128, 1) coarse_tc_kernel(const __grid_constant__ CoarseParams p) {
+  using S = TcShape<KIND, D>;
+  using namespace ptx;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t full[2], empty[2], done;
+  __shared__ uint32_t tmem_base;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int C = p.C, BH = p.BH;
+  const int m0 = blockIdx.x * 128, n0 = blockIdx.y * S::NT, bh = blockIdx.z;
+  const int K = KIND == 0 ? D : p.Cp;
+  const int nch = (K + 63) / 64;
+  const uint64_t lim = p.wait_ns;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
     }
+    mbar_init(&done, 1);
+    fence_mbar_init();
   }
-  if (S == 1) {
-    if (p.oc_copy) {
+  if (warp == 0) {
+    tmem_alloc(&tmem_base, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+  auto a_tile = [&](int st, int t) { return tiles + st * S::STAGE + t * S::A_BYTES; };
+  auto b_tile = [&](int st, int t) { return tiles + st * S::STAGE + 3 * S::A_BYTES + t * S::B_BYTES; };
+
+  if (warp == 0 && lane == 0) {
+    const CUtensorMap* ta = KIND == 0 ? &p.tm_qs : &p.tm_ps;
+    const CUtensorMap* tb = KIND == 0 ? &p.tm_ks : &p.tm_vs;
+    int armed = 0;
+    for (int c = 0; c < nch; ++c) {
+      const int st = c & 1;
+      if (c >= 2 && !mbar_wait(&empty[st], ((c >> 1) - 1) & 1, lim)) {
+        atomicOr(p.err, kErrTimeout);
+        break;
+      }
+      mbar_arrive_expect_tx(&full[st], S::STAGE);
+      ++armed;
+      for (int t = 0; t < 3; ++t) {
+        tma_load_3d(a_tile(st, t), ta, &full[st], 64 * c, m0, t * BH + bh);
+        if (KIND == 0) {
+          tma_load_3d(b_tile(st, t), tb, &full[st], 64 * c, n0, t * BH + bh);
+        } else {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int r = m0 + tile_row(i);
-        if (r >= C) continue;
-#pragma unroll
-        for (int jb = 0; jb < 8; jb += 4) {
-          const int c = tile_col(jb);
-          if (c < D) *reinterpret_cast<float4*>(p.oc_copy + ((size_t)bh * C + r) * D + c) =
-                         make_float4(acc[i][jb], acc[i][jb + 1], acc[i][jb + 2], acc[i][jb + 3]);
+          for (int h = 0; h < D / 64; ++h) tma_load_3d(b_tile(st, t) + h * 8192, tb, &full[st], 64 * h, 64 * c, t * BH + bh);
         }
       }
     }
-    return;
-  }
-  __threadfence();
-  __syncthreads();
-  int* cnt = p.tile_cnt + bh * gridDim.x + mt;
-  if (threadIdx.x == 0) last = (atomicAdd(cnt, 1) == S - 1);
-  __syncthreads();
-  if (!last) return;
-  __threadfence();
-  // Sum the partials of the tile's rows in split order (16 bytes per thread per step).
-  const int rows = min(kGM, C - m0), vecs = rows * (D / 4);
-  for (int v = threadIdx.x; v < vecs; v += kGThreads) {
-    const size_t o = ((size_t)bh * C + m0 + v / (D / 4)) * D + (v % (D / 4)) * 4;
-    float4 t = __ldcg(reinterpret_cast<const float4*>(p.opart + o));
-    for (int s2 = 1; s2 < S; ++s2) {
-      const float4 u = __ldcg(reinterpret_cast<const float4*>(p.opart + (size_t)s2 * p.BH * C * D + o));
-      t.x += u.x; t.y += u.y; t.z += u.z; t.w += u.w;
+    // Drain: the last armed phase of each stage covers all copies issued.
+    for (int st = 0; st < 2 && st < armed; ++st) mbar_wait(&full[st], (((armed - 1 - st) >> 1)) & 1, lim);
+  } else if (warp == 1 && lane == 0) {
+    constexpr uint32_t idesc = idesc_bf16_f32(128, S::NT, false, KIND == 1);
+    // Term pairs (A term, B term) of the six products kept.
+    constexpr int pa[6] = {2, 0, 1, 1, 0, 0}, pb[6] = {0, 2, 1, 0, 1, 0};
+    bool ok = true;
+    for (int c = 0; c < nch && ok; ++c) {
+      const int st = c & 1;
+      if (!mbar_wait(&full[st], (c >> 1) & 1, lim)) {
+        atomicOr(p.err, kErrTimeout);
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+        for (int q = 0; q < 6; ++q) {
+          const uint64_t ad = sdesc_sw128(smem_u32(a_tile(st, pa[q])), 16, 1024) + (uint64_t)((kk * 32) >> 4);
+          uint64_t bd;
+          if (KIND == 0) bd = sdesc_sw128(smem_u32(b_tile(st, pb[q])), 16, 1024) + (uint64_t)((kk * 32) >> 4);
+          else bd = sdesc_sw128(smem_u32(b_tile(st, pb[q])), 8192, 1024) + (uint64_t)((kk * 2048) >> 4);
+          mma_bf16_ss(tmem, ad, bd, idesc, (c > 0 || kk > 0 || q > 0) ? 1u : 0u);
+        }
+      mma_commit(&empty[st]);
     }
-    *reinterpret_cast<float4*>(p.oc + o) = t;
-    if (p.oc_copy) *reinterpret_cast<float4*>(p.oc_copy + o) = t;
+    mma_commit(&done);
   }
-  if (threadIdx.x == 0) *cnt = 0;  // ready for the next run
+  __syncwarp();
+  // Epilogue: warp w holds accumulator rows 32 w .. 32 w + 31 (one per thread).
+  const bool have = mbar_wait(&done, 0, lim);
+  if (!have && lane == 0) atomicOr(p.err, kErrTimeout);
+  tc_fence_after();
+  const int row = m0 + 32 * warp + lane;
+#pragma unroll
+  for (int cg = 0; cg < S::NT / 32; ++cg) {
+    uint32_t r[32];
+    tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16) + 32 * cg, r);
+    tmem_wait_ld();
+    if (!have || row >= C) continue;
+    if (KIND == 0) {
+      float* dst = p.s + ((size_t)bh * C + row) * C + n0 + 32 * cg;
+      const int ncol = min(32, C - (n0 + 32 * cg));
+      if ((C & 3) == 0 && ncol == 32) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(dst + e) =
+              make_float4(__uint_as_float(r[e]) * p.scale, __uint_as_float(r[e + 1]) * p.scale,
+                          __uint_as_float(r[e + 2]) * p.scale, __uint_as_float(r[e + 3]) * p.scale);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          if (e < ncol) dst[e] = __uint_as_float(r[e]) * p.scale;
+      }
+    } else {
+      const size_t o = ((size_t)bh * C + row) * D + 32 * cg;
+#pragma unroll
+      for (int e = 0; e < 32; e += 4) {
+        const float4 v = make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]), __uint_as_float(r[e + 2]),
+                                     __uint_as_float(r[e + 3]));
+        *reinterpret_cast<float4*>(p.oc + o + e) = v;
+        if (p.oc_copy) *reinterpret_cast<float4*>(p.oc_copy + o + e) = v;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+template <int KIND, int D>
+cudaError_t launch_tc(const CoarseParams& p, cudaStream_t st) {
+  using S = TcShape<KIND, D>;
+  cudaError_t e = cudaFuncSetAttribute(coarse_tc_kernel<KIND, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((p.C + 127) / 128, KIND == 0 ? (p.C + 127) / 128 : 1, p.BH);
+  coarse_tc_kernel<KIND, D><<<grid, 128, S::SMEM, st>>>(p);
+  return cudaGetLastError();
 }
 
 template <int PER>
@@ -486,9 +455,7 @@ cudaError_t launch_select(const CoarseParams& p, cudaStream_t st) {
 }  // namespace
 
 cudaError_t launch_coarse(const CoarseParams& p, cudaStream_t st) {
-  const int mtiles = (p.C + kGM - 1) / kGM, ntiles = (p.C + kGN - 1) / kGN;
-  coarse_scores_kernel<<<dim3(ntiles, mtiles, p.BH), kGThreads, 0, st>>>(p);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = p.D == 128 ? launch_tc<0, 128>(p, st) : launch_tc<0, 64>(p, st);
   if (e != cudaSuccess) return e;
   const int per = (p.C + 31) / 32;
   if (per <= 1) e = launch_select<1>(p, st);
@@ -504,8 +471,7 @@ cudaError_t launch_coarse(const CoarseParams& p, cudaStream_t st) {
   else if (per <= 96) e = launch_select<96>(p, st);
   else e = launch_select<128>(p, st);
   if (e != cudaSuccess) return e;
-  coarse_output_kernel<<<dim3(mtiles, p.splits, p.BH), kGThreads, 0, st>>>(p);
-  return cudaGetLastError();
+  return p.D == 128 ? launch_tc<1, 128>(p, st) : launch_tc<1, 64>(p, st);
 }
 
 }  // namespace vsa

@@ -68,6 +68,29 @@ __global__ void __launch_bounds__(256) gather_pool_kernel(const GatherParams p) 
     const float inv = 1.0f / kCube;
     *reinterpret_cast<float4*>(pool) = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
     *reinterpret_cast<float4*>(pool + 4) = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+    // The same means as three bf16 terms (hi, mid, lo) for the tensor-core
+    // coarse products, packed two per 32-bit word (lower element in the low half).
+    uint32_t w[3][4];
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+      float x[2] = {acc[e] * inv, acc[e + 1] * inv};
+      __nv_bfloat162 h[3];
+#pragma unroll
+      for (int k = 0; k < 3; ++k) {
+        h[k] = __floats2bfloat162_rn(x[0], x[1]);
+        const float2 back = __bfloat1622float2(h[k]);
+        x[0] -= back.x;
+        x[1] -= back.y;
+      }
+#pragma unroll
+      for (int k = 0; k < 3; ++k) w[k][e / 2] = (uint32_t)__bfloat16_as_ushort(h[k].x) |
+                                               ((uint32_t)__bfloat16_as_ushort(h[k].y) << 16);
+    }
+    const size_t plane = (size_t)p.BH * p.C * D;
+    __nv_bfloat16* sp = p.split[tensor] + ((size_t)bh * p.C + c) * D + chunk * 8;
+#pragma unroll
+    for (int k = 0; k < 3; ++k)
+      *reinterpret_cast<uint4*>(sp + k * plane) = make_uint4(w[k][0], w[k][1], w[k][2], w[k][3]);
   }
 }
 

@@ -25,19 +25,23 @@ struct GatherParams {
   const __nv_bfloat16* src[3];  // q, k, v raster [BH, N, D]
   __nv_bfloat16* dst[3];        // cube-major [BH, C, 64, D]; null: pool only for that tensor
   float* pool[3];               // [BH, C, D] cube means
+  __nv_bfloat16* split[3];      // [3, BH, C, D] the means as three bf16 terms (hi, mid, lo)
   int BH, C, H, W, N;
 };
 
 struct CoarseParams {
-  const float* qpool;  // [BH, C, D]
-  const float* kpool;
-  const float* vpool;
-  float* s;            // [BH, C, C] scores, then probabilities
+  // 3-D maps (128-byte swizzle) over the bf16 three-term splits:
+  //   tm_qs, tm_ks: [3 * BH][C][D], boxes of 128 rows x 64 channels;
+  //   tm_vs: [3 * BH][C][D], boxes of 64 rows x 64 channels;
+  //   tm_ps: [3 * BH][C][Cp], boxes of 128 rows x 64 columns.
+  CUtensorMap tm_qs, tm_ks, tm_vs, tm_ps;
+  float* s;            // [BH, C, C] scores
+  __nv_bfloat16* psplit;  // [3, BH, C, Cp] coarse probabilities as three bf16 terms
   float* oc;           // [BH, C, D]
   float* oc_copy;      // optional second destination of oc (may be null)
-  float* opart;        // [splits, BH, C, D] partial products of the output GEMM
-  int* tile_cnt;       // [BH, ceil(C/64)] arrival counts (zero between runs)
-  int splits;          // K splits of the output GEMM (1: no partials)
+  int Cp;              // C rounded up to a multiple of 8 (row pitch of psplit)
+  int* err;
+  unsigned long long wait_ns;
   int32_t* idx;        // [BH, C, kcap]
   int32_t* cnt;        // [BH, C]
   int BH, C, D, kcap;

@@ -38,7 +38,7 @@ class Config(ctypes.Structure):
 
 class WorkspaceLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in ("q_cube", "k_cube", "v_cube", "q_pool", "k_pool", "v_pool",
-                                               "o_coarse", "s_coarse", "o_part", "tile_cnt", "cnt", "err",
+                                               "o_coarse", "s_coarse", "pool_split", "p_split", "cnt", "err",
                                                "total")]
 
 
