@@ -220,6 +220,124 @@ __device__ __forceinline__ bool topk_small(const uint32_t (&key)[PER], int C, in
   return true;
 }
 
+// Fixed top-K <= 32 with the row's keys in shared memory instead of
+// registers, so more warps (rows) per SM hide the latency of the warp-wide
+// reductions. One warp per row; per warp the shared memory holds the keys
+// (C rounded up to 32) and kCandCap candidate ids. Passes: load the scores as
+// keys (lane maxima of score and key), the row sum, the probabilities as three
+// bf16 terms, then the selection through the candidates at or above the
+// lane-maxima bound, compacted in place; more than kCandCap candidates fall
+// back to the bit search over all keys.
+__global__ void __launch_bounds__(256, 4) coarse_select_small_kernel(const CoarseParams p) {
+  extern __shared__ __align__(16) uint8_t dyn[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 8 + warp;
+  if (row >= p.BH * p.C) return;
+  const int C = p.C, Kt = p.topk;
+  const int stride = (C + 31) / 32 * 32;
+  uint32_t* keys = reinterpret_cast<uint32_t*>(dyn) + (size_t)warp * (stride + kCandCap);
+  int* cidx = reinterpret_cast<int*>(keys + stride);
+  const float* srow = p.s + (size_t)row * C;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+
+  float lm = -INFINITY;
+  uint32_t lkmax = 0;
+  for (int j0 = 0; j0 < C; j0 += 256) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = j0 + lane + 32 * u;
+      v[u] = j < C ? srow[j] : -INFINITY;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = j0 + lane + 32 * u;
+      if (j < C) {
+        const uint32_t k = order_key(v[u]);
+        keys[j] = k;
+        lkmax = max(lkmax, k);
+        lm = fmaxf(lm, v[u]);
+      }
+    }
+  }
+  const float m = warp_max(lm);
+  const float mb = m * kLog2e;
+  __syncwarp();
+  float l = 0.f;
+  for (int j = lane; j < C; j += 32) l += fast_exp2(fmaf(key_value(keys[j]), kLog2e, -mb));
+  l = warp_sum(l);
+  // Probabilities as three bf16 terms (zero in the padding columns C .. Cp-1).
+  const float inv_l = 1.0f / l;
+  const size_t plane = (size_t)p.BH * C * p.Cp;
+  __nv_bfloat16* prow = p.psplit + (size_t)row * p.Cp;
+  for (int j = lane; j < p.Cp; j += 32) {
+    const float x = j < C ? fast_exp2(fmaf(key_value(keys[j]), kLog2e, -mb)) * inv_l : 0.f;
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    const float r1 = x - __bfloat162float(h);
+    const __nv_bfloat16 md = __float2bfloat16_rn(r1);
+    prow[j] = h;
+    prow[plane + j] = md;
+    prow[2 * plane + j] = __float2bfloat16_rn(r1 - __bfloat162float(md));
+  }
+  if (!p.do_select) return;
+  int32_t* irow = p.idx + (size_t)row * p.kcap;
+  // Lower bound lo of the Kt-th largest key (Kt <= 32 and every lane with a key
+  // holds one at or above it) and the row maximum hi.
+  const uint32_t lo = __reduce_min_sync(0xffffffffu, lane < C ? lkmax : 0xffffffffu);
+  const uint32_t hi = __reduce_max_sync(0xffffffffu, lkmax);
+  unsigned nl = 0;
+  for (int j = lane; j < C; j += 32) nl += (keys[j] >= lo);
+  const int n = (int)__reduce_add_sync(0xffffffffu, nl);
+  if (n <= kCandCap) {
+    // In-place compaction in ascending id order: a candidate never lands past
+    // the position it is read from, and every lane reads before the ballot.
+    int pos = 0;
+    for (int j0 = 0; j0 < C; j0 += 32) {
+      const int j = j0 + lane;
+      const uint32_t k = j < C ? keys[j] : 0u;
+      const bool t = j < C && k >= lo;
+      const unsigned tb = __ballot_sync(0xffffffffu, t);
+      if (t) {
+        const int q = pos + __popc(tb & lt_mask);
+        keys[q] = k;
+        cidx[q] = j;
+      }
+      pos += __popc(tb);
+    }
+    __syncwarp();
+    if (n <= 32) topk_from_candidates<1>(keys, cidx, n, Kt, lo, hi, irow);
+    else if (n <= 64) topk_from_candidates<2>(keys, cidx, n, Kt, lo, hi, irow);
+    else if (n <= 128) topk_from_candidates<4>(keys, cidx, n, Kt, lo, hi, irow);
+    else topk_from_candidates<8>(keys, cidx, n, Kt, lo, hi, irow);
+  } else {
+    // Bit search for the Kt-th largest key over all keys, then the ids above it
+    // and the lowest-id ones equal to it, ascending.
+    uint32_t T = 0;
+    for (int b = 31; b >= 0; --b) {
+      const uint32_t c = T | (1u << b);
+      unsigned cnt = 0;
+      for (int j = lane; j < C; j += 32) cnt += (keys[j] >= c);
+      if ((int)__reduce_add_sync(0xffffffffu, cnt) >= Kt) T = c;
+    }
+    unsigned gt = 0;
+    for (int j = lane; j < C; j += 32) gt += (keys[j] > T);
+    const int need = Kt - (int)__reduce_add_sync(0xffffffffu, gt);
+    int pos = 0, eq_seen = 0;
+    for (int j0 = 0; j0 < C; j0 += 32) {
+      const int j = j0 + lane;
+      const uint32_t k = j < C ? keys[j] : 0u;
+      const bool is_eq = j < C && k == T;
+      const unsigned eqb = __ballot_sync(0xffffffffu, is_eq);
+      const bool take = (j < C && k > T) || (is_eq && eq_seen + __popc(eqb & lt_mask) < need);
+      const unsigned tb = __ballot_sync(0xffffffffu, take);
+      if (take) irow[pos + __popc(tb & lt_mask)] = j;
+      pos += __popc(tb);
+      eq_seen += __popc(eqb);
+    }
+  }
+  if (lane == 0) p.cnt[row] = Kt;
+}
+
 // TOPK: fixed top-K (no top-p scratch, fewer registers, more warps per SM).
 template <int PER, bool TOPK>
 __global__ void __launch_bounds__(256, TOPK ? 3 : 1) coarse_select_kernel(const CoarseParams p) {
@@ -536,6 +654,16 @@ cudaError_t launch_tc(const CoarseParams& p, cudaStream_t st) {
 template <int PER>
 cudaError_t launch_select(const CoarseParams& p, cudaStream_t st) {
   const int rows = p.BH * p.C;
+  if (p.topk > 0 && p.topk <= 32) {
+    const size_t smem = (size_t)8 * ((p.C + 31) / 32 * 32 + kCandCap) * 4;
+    if (smem > 48 * 1024) {
+      cudaError_t e = cudaFuncSetAttribute(coarse_select_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)smem);
+      if (e != cudaSuccess) return e;
+    }
+    coarse_select_small_kernel<<<(rows + 7) / 8, 256, smem, st>>>(p);
+    return cudaGetLastError();
+  }
   if (!p.do_select || p.topk > 0) {
     coarse_select_kernel<PER, true><<<(rows + 7) / 8, 256, 0, st>>>(p);
     return cudaGetLastError();
