@@ -183,3 +183,39 @@ def test_out_of_range_index_is_reported_not_read():
     o2, i2, _ = plan.run(*dev_in)
     plan.check()
     assert torch.equal(o2, out)
+
+
+@pytest.mark.parametrize("wl", [SMALL[1], SMALL[6]], ids=["cube_k5_odd", "d64_k7"])
+def test_coarse_scores_keep_fp32_accuracy(wl):
+    """The coarse products run on the tensor cores with every fp32 operand
+    written as three bf16 terms; the scores must stay at fp32 accuracy (a
+    single bf16 term would be off by ~1e-3)."""
+    inputs = synth.make_inputs(wl)
+    plan, dev_in, out, idx, cnt = _run(wl, inputs)
+    q, k, v, gc, gf = inputs
+    BH = wl.B * wl.heads
+    s_gpu = plan.workspace_view("s_coarse", torch.float32, (BH, wl.C, wl.C)).cpu().numpy()
+    for b in range(wl.B):
+        for h in range(wl.heads):
+            r = oracle_head(wl, q, k, v, gc, gf, b, h)
+            assert_close(s_gpu[b * wl.heads + h], r["s"], "coarse scores", max_abs=1e-5, mean_abs=1e-6)
+
+
+@pytest.mark.parametrize("T,H,W_", [(8, 32, 32), (16, 32, 48)], ids=["C128_candidates", "C384_fallback"])
+def test_all_equal_scores_select_lowest_ids(T, H, W_):
+    """q = 0 makes every coarse score equal: top-K must take cubes 0..K-1 in
+    every row (ties to the lower id). With C = 384 every score is a candidate
+    above the lane-maxima bound (more than 256), which exercises the full bit
+    search of the shared-memory select kernel."""
+    wl = W["tiny"].with_(name="zero_q", heads=1, D=64, T=T, H=H, W=W_, topk=8)
+    q, k, v, gc, gf = synth.make_inputs(wl)
+    q = torch.zeros_like(q)
+    plan, dev_in, out, idx, cnt = _run(wl, (q, k, v, gc, gf))
+    idx_h, cnt_h = idx.cpu().numpy(), cnt.cpu().numpy()
+    assert (cnt_h == 8).all()
+    assert (idx_h[0, 0] == np.arange(8, dtype=np.int32)[None, :]).all()
+    sample = np.array([0, 1, wl.C // 2, wl.C - 1])
+    r = oracle_head(wl, q, k, v, gc, gf, 0, 0, query_cubes=sample)
+    perm = oracle.cube_perm(wl.T, wl.H, wl.W)
+    toks = perm.reshape(wl.C, 64)[sample].reshape(-1)
+    assert_close(out[0, 0].float().cpu().numpy()[toks], r["out"][toks], "output, all-equal scores")
