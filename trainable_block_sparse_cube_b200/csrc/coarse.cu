@@ -176,50 +176,6 @@ __device__ __forceinline__ void topk_from_candidates(const uint32_t* ckey, const
   }
 }
 
-// Top-K selection of a row for Kt <= 32 through the candidates at or above
-// lo = the minimum of the lanes' maxima (a lower bound of the Kt-th largest
-// key). Returns false, writing nothing, when there are more than kCandCap.
-template <int PER>
-__device__ __forceinline__ bool topk_small(const uint32_t (&key)[PER], int C, int Kt, uint32_t* ckey, int* cidx,
-                                           int32_t* irow) {
-  const int lane = threadIdx.x & 31;
-  const uint32_t lt_mask = (1u << lane) - 1u;
-  uint32_t lmax = 0;
-  bool any = false;
-#pragma unroll
-  for (int u = 0; u < PER; ++u)
-    if (lane + 32 * u < C) {
-      lmax = max(lmax, key[u]);
-      any = true;
-    }
-  const uint32_t lo = __reduce_min_sync(0xffffffffu, any ? lmax : 0xffffffffu);
-  const uint32_t hi = __reduce_max_sync(0xffffffffu, lmax);
-  unsigned nl = 0;
-#pragma unroll
-  for (int u = 0; u < PER; ++u) nl += (key[u] >= lo);
-  const int n = (int)__reduce_add_sync(0xffffffffu, nl);
-  if (n > kCandCap) return false;
-  int pos = 0;
-#pragma unroll
-  for (int u = 0; u < PER; ++u) {
-    const bool t = key[u] >= lo;
-    const unsigned tb = __ballot_sync(0xffffffffu, t);
-    if (t) {
-      const int q = pos + __popc(tb & lt_mask);
-      ckey[q] = key[u];
-      cidx[q] = lane + 32 * u;
-    }
-    pos += __popc(tb);
-  }
-  __syncwarp();
-  if (n <= 32) topk_from_candidates<1>(ckey, cidx, n, Kt, lo, hi, irow);
-  else if (n <= 64) topk_from_candidates<2>(ckey, cidx, n, Kt, lo, hi, irow);
-  else if (n <= 128) topk_from_candidates<4>(ckey, cidx, n, Kt, lo, hi, irow);
-  else topk_from_candidates<8>(ckey, cidx, n, Kt, lo, hi, irow);
-  __syncwarp();
-  return true;
-}
-
 // Fixed top-K <= 32 with the row's keys in shared memory instead of
 // registers, so more warps (rows) per SM hide the latency of the warp-wide
 // reductions. One warp per row; per warp the shared memory holds the keys
@@ -338,12 +294,12 @@ __global__ void __launch_bounds__(256, 4) coarse_select_small_kernel(const Coars
   if (lane == 0) p.cnt[row] = Kt;
 }
 
-// TOPK: fixed top-K (no top-p scratch, fewer registers, more warps per SM).
+// Register-resident selection for top-K > 32 and top-p (TOPK: fixed top-K,
+// no top-p scratch, fewer registers).
 template <int PER, bool TOPK>
 __global__ void __launch_bounds__(256, TOPK ? 3 : 1) coarse_select_kernel(const CoarseParams p) {
   extern __shared__ __align__(16) uint8_t dyn[];
   __shared__ uint32_t cand_all[8][kCandCap];
-  __shared__ int cand_idx[TOPK ? 8 : 1][kCandCap];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * 8 + warp;
   if (row >= p.BH * p.C) return;
@@ -368,10 +324,7 @@ __global__ void __launch_bounds__(256, TOPK ? 3 : 1) coarse_select_kernel(const 
     if (lane + 32 * u < C) l += fast_exp2(fmaf(key_value(key[u]), kLog2e, -mb));
   l = warp_sum(l);
 
-  const bool small_done = TOPK && p.do_select && p.topk <= 32 &&
-                          topk_small<PER>(key, C, p.topk, cand_all[warp], cand_idx[TOPK ? warp : 0],
-                                          p.idx + (size_t)row * p.kcap);
-  if (p.do_select && !small_done) {
+  if (p.do_select) {
     const int Kt = p.topk > 0 ? p.topk : p.kmax;
     // T is the Kt-th largest key exactly.
     const uint32_t T = kth_largest<PER>(key, C, Kt, cand_all[warp]);
@@ -470,8 +423,6 @@ __global__ void __launch_bounds__(256, TOPK ? 3 : 1) coarse_select_kernel(const 
     }
     for (int c = n_out + lane; c < p.kcap; c += 32) irow[c] = -1;
     if (lane == 0) p.cnt[row] = n_out;
-  } else if (small_done && lane == 0) {
-    p.cnt[row] = p.topk;
   }
   // Probabilities over the scores as three bf16 terms (zero in the padding
   // columns C .. Cp-1), the A operand of the output product.
