@@ -125,6 +125,29 @@ vsa_status vsa_run_fixed_idx(vsa_plan_t plan, const void* q, const void* k, cons
                              const float* gate_f, const int32_t* idx_in, const int32_t* cnt_in, void* out,
                              float* out_coarse, float* out_fine, void* stream);
 
+/* Forward pass on HOST buffers: copies the inputs to the device, runs the
+ * forward pass (as vsa_run) and copies the results back, all enqueued on
+ * `stream`. The pages describing the method have no counterpart of this
+ * entry point; it is the path for callers whose tensors live in host memory.
+ * The work is split by (batch, head): the copy of slice i+1 to the device
+ * and of slice i-1 back to the host run on two library streams while slice
+ * i is computed on `stream`, so the copies overlap the computation (and
+ * each other) when the host buffers are pinned (page-locked); pageable
+ * buffers work too, without overlap.
+ *   q, k, v: [B,heads,N,D] bf16 host; gate_c, gate_f: [B,heads,N] fp32 host;
+ *   out: [B,heads,N,D] bf16 host (written); idx: [B,heads,C,Kcap] int32 host
+ *   (written); cnt: [B,heads,C] int32 host (written) or NULL.
+ * The host results are complete once `stream` has reached the end of the
+ * call's work (synchronise it before reading them). The first call on a plan
+ * allocates device copies of the inputs and results (B*heads*(5*N*D*2 +
+ * 2*N*4 + C*Kcap*4 + C*4) bytes, rounded up), a workspace for one
+ * (batch, head) slice and two streams; later calls allocate nothing and the
+ * plan releases them in vsa_plan_destroy. Device-side errors are reported by
+ * vsa_check(plan). Returns VSA_ERR_INVALID_ARG for a NULL argument (other
+ * than cnt) and VSA_ERR_CUDA if a copy, an allocation or a launch fails. */
+vsa_status vsa_run_host(vsa_plan_t plan, const void* q, const void* k, const void* v, const float* gate_c,
+                        const float* gate_f, void* out, int32_t* idx, int32_t* cnt, void* stream);
+
 /* One-call form. Keeps a library-owned plan and workspace per distinct
  * configuration (the first call for a configuration allocates device memory
  * with cudaMalloc; later calls allocate nothing). topk > 0 selects top-K;

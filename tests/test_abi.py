@@ -91,6 +91,7 @@ def test_plan_argument_errors(lib):
     assert lib.vsa_plan(ctypes.byref(h), ctypes.byref(c), ctypes.c_void_p((1 << 20) + 16), 1 << 30) == 4
     assert lib.vsa_plan(ctypes.byref(h), ctypes.byref(c), ctypes.c_void_p(1 << 20), 16) == 1
     assert lib.vsa_run(None, *([None] * 9)) == 1
+    assert lib.vsa_run_host(None, *([None] * 9)) == 1
     assert lib.vsa_check(None) == 1
     assert lib.vsa_set_wait_limit_ns(None, 10 ** 9) == 1
     assert lib.vsa_set_debug_stall(None, 1) == 1

@@ -219,3 +219,22 @@ def test_all_equal_scores_select_lowest_ids(T, H, W_):
     perm = oracle.cube_perm(wl.T, wl.H, wl.W)
     toks = perm.reshape(wl.C, 64)[sample].reshape(-1)
     assert_close(out[0, 0].float().cpu().numpy()[toks], r["out"][toks], "output, all-equal scores")
+
+
+@pytest.mark.parametrize("wl", [SMALL[2], SMALL[5]], ids=["cube_b2", "tiny_topp_d64"])
+def test_host_buffers_match_device_run(wl):
+    """vsa_run_host (pinned host tensors in and out, per-(batch, head) slices
+    pipelined over copy streams) returns exactly what vsa_run returns on the
+    same inputs in device memory."""
+    inputs = synth.make_inputs(wl)
+    plan, dev_in, out, idx, cnt = _run(wl, inputs)
+    hin = [t.pin_memory() for t in inputs]
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    hidx = torch.full(idx.shape, -5, dtype=idx.dtype).pin_memory()
+    hcnt = torch.full(cnt.shape, -5, dtype=cnt.dtype).pin_memory()
+    for _ in range(2):  # the second call reuses the device copies and streams
+        plan.run_host(*hin, hout, hidx, hcnt)
+        plan.check()
+        assert torch.equal(hout, out.cpu()) and torch.equal(hidx, idx.cpu()) and torch.equal(hcnt, cnt.cpu())
+        hout.zero_()
+        hidx.fill_(-5)

@@ -12,6 +12,21 @@
 #include "../../include/vsa.h"
 #include "vsa_common.cuh"
 
+// State of vsa_run_host, created by its first call on a plan: device copies
+// of the inputs and results, a plan (and workspace) over one (batch, head)
+// slice, two copy streams and the events that chain the slices.
+struct HostPath {
+  vsa_plan_s* sub;
+  void* sub_ws;
+  char* dbuf;       // device copies: q, k, v, gate_c, gate_f, out, idx, cnt
+  size_t off[8];    // offsets of the eight arrays in dbuf
+  size_t slice[8];  // bytes of one (batch, head) slice of each
+  cudaStream_t s_in, s_out;
+  cudaEvent_t e_start, e_end;
+  cudaEvent_t* e_in;   // per slice: inputs on the device
+  cudaEvent_t* e_out;  // per slice: results on the device
+};
+
 struct vsa_plan_s {
   vsa_config cfg;
   int BH, N, C, kcap;
@@ -31,6 +46,7 @@ struct vsa_plan_s {
   int timing;        // record stage events
   int timed_runs;    // runs recorded since timing was enabled
   cudaEvent_t ev[4];
+  HostPath* host;    // vsa_run_host state (null until its first call)
 };
 
 namespace {
@@ -259,6 +275,29 @@ vsa_status run_common(vsa_plan_t P, const void* q, const void* k, const void* v,
 
 }  // namespace
 
+// Releases vsa_run_host state (waits for its streams first).
+static void host_path_free(HostPath* H) {
+  if (!H) return;
+  if (H->s_in) cudaStreamSynchronize(H->s_in);
+  if (H->s_out) cudaStreamSynchronize(H->s_out);
+  if (H->sub) vsa_plan_destroy(H->sub);
+  if (H->sub_ws) cudaFree(H->sub_ws);
+  if (H->dbuf) cudaFree(H->dbuf);
+  if (H->e_in) {
+    for (int i = 0; H->e_in[i]; ++i) cudaEventDestroy(H->e_in[i]);
+    delete[] H->e_in;
+  }
+  if (H->e_out) {
+    for (int i = 0; H->e_out[i]; ++i) cudaEventDestroy(H->e_out[i]);
+    delete[] H->e_out;
+  }
+  if (H->e_start) cudaEventDestroy(H->e_start);
+  if (H->e_end) cudaEventDestroy(H->e_end);
+  if (H->s_in) cudaStreamDestroy(H->s_in);
+  if (H->s_out) cudaStreamDestroy(H->s_out);
+  delete H;
+}
+
 extern "C" {
 
 size_t vsa_workspace_bytes(const vsa_config* cfg) {
@@ -329,6 +368,83 @@ vsa_status vsa_run_fixed_idx(vsa_plan_t plan, const void* q, const void* k, cons
                              float* out_coarse, float* out_fine, void* stream) {
   return run_common(plan, q, k, v, gate_c, gate_f, false, idx_in, cnt_in, nullptr, nullptr, out, out_coarse, out_fine,
                     stream);
+}
+
+vsa_status vsa_run_host(vsa_plan_t plan, const void* q, const void* k, const void* v, const float* gate_c,
+                        const float* gate_f, void* out, int32_t* idx, int32_t* cnt, void* stream) {
+  if (!plan || !q || !k || !v || !gate_c || !gate_f || !out || !idx) return VSA_ERR_INVALID_ARG;
+  const int n = plan->BH;
+  HostPath* H = plan->host;
+  if (!H) {
+    H = new (std::nothrow) HostPath();
+    if (!H) return VSA_ERR_INVALID_ARG;
+    plan->host = H;
+    vsa_config sc = plan->cfg;
+    sc.B = 1;
+    sc.heads = 1;
+    const size_t sb = vsa_workspace_bytes(&sc);
+    const size_t nd2 = (size_t)plan->N * plan->cfg.D * 2, n4 = (size_t)plan->N * 4;
+    const size_t sl[8] = {nd2, nd2, nd2, n4, n4, nd2, (size_t)plan->C * plan->kcap * 4, (size_t)plan->C * 4};
+    size_t total = 0;
+    for (int a = 0; a < 8; ++a) {
+      H->slice[a] = sl[a];
+      H->off[a] = total;
+      total += align_up(sl[a] * n, 256);
+    }
+    H->e_in = new (std::nothrow) cudaEvent_t[n + 1]();
+    H->e_out = new (std::nothrow) cudaEvent_t[n + 1]();
+    bool ok = sb > 0 && H->e_in && H->e_out && cudaMalloc(&H->sub_ws, sb) == cudaSuccess &&
+              cudaMalloc(reinterpret_cast<void**>(&H->dbuf), total) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&H->s_in, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&H->s_out, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&H->e_start, cudaEventDisableTiming) == cudaSuccess &&
+              cudaEventCreateWithFlags(&H->e_end, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; ok && i < n; ++i)
+      ok = cudaEventCreateWithFlags(&H->e_in[i], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&H->e_out[i], cudaEventDisableTiming) == cudaSuccess;
+    vsa_status ps = ok ? vsa_plan(&H->sub, &sc, H->sub_ws, sb) : VSA_ERR_CUDA;
+    if (ps != VSA_OK) {
+      host_path_free(H);
+      plan->host = nullptr;
+      return ps;
+    }
+  }
+  H->sub->wait_ns = plan->wait_ns;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // The copies start after the work already on `stream`; `stream` resumes
+  // after the last copy back.
+  if (cudaEventRecord(H->e_start, st) != cudaSuccess || cudaStreamWaitEvent(H->s_in, H->e_start, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(H->s_out, H->e_start, 0) != cudaSuccess)
+    return VSA_ERR_CUDA;
+  const void* hin[5] = {q, k, v, gate_c, gate_f};
+  void* hres[3] = {out, idx, cnt};
+  for (int i = 0; i < n; ++i) {
+    // slice i in: copy stream 1
+    for (int a = 0; a < 5; ++a)
+      if (cudaMemcpyAsync(H->dbuf + H->off[a] + i * H->slice[a], static_cast<const char*>(hin[a]) + i * H->slice[a],
+                          H->slice[a], cudaMemcpyHostToDevice, H->s_in) != cudaSuccess)
+        return VSA_ERR_CUDA;
+    if (cudaEventRecord(H->e_in[i], H->s_in) != cudaSuccess || cudaStreamWaitEvent(st, H->e_in[i], 0) != cudaSuccess)
+      return VSA_ERR_CUDA;
+    // slice i forward: `stream`
+    char* d[8];
+    for (int a = 0; a < 8; ++a) d[a] = H->dbuf + H->off[a] + i * H->slice[a];
+    const vsa_status rs = vsa_run(H->sub, d[0], d[1], d[2], reinterpret_cast<float*>(d[3]),
+                                  reinterpret_cast<float*>(d[4]), d[5], reinterpret_cast<int32_t*>(d[6]),
+                                  reinterpret_cast<int32_t*>(d[7]), stream);
+    if (rs != VSA_OK) return rs;
+    if (cudaEventRecord(H->e_out[i], st) != cudaSuccess || cudaStreamWaitEvent(H->s_out, H->e_out[i], 0) != cudaSuccess)
+      return VSA_ERR_CUDA;
+    // slice i out: copy stream 2
+    for (int a = 5; a < 8; ++a)
+      if (hres[a - 5] && cudaMemcpyAsync(static_cast<char*>(hres[a - 5]) + i * H->slice[a], d[a], H->slice[a],
+                                         cudaMemcpyDeviceToHost, H->s_out) != cudaSuccess)
+        return VSA_ERR_CUDA;
+  }
+  if (cudaEventRecord(H->e_end, H->s_out) != cudaSuccess || cudaStreamWaitEvent(st, H->e_end, 0) != cudaSuccess)
+    return VSA_ERR_CUDA;
+  plan->last_stream = st;
+  return VSA_OK;
 }
 
 namespace {
@@ -460,6 +576,10 @@ vsa_status vsa_forward_noalloc(const void* q, const void* k, const void* v, cons
 
 vsa_status vsa_check(vsa_plan_t plan) {
   if (!plan) return VSA_ERR_INVALID_ARG;
+  if (plan->host && plan->host->sub) {
+    const vsa_status hs = vsa_check(plan->host->sub);
+    if (hs != VSA_OK) return hs;
+  }
   if (cudaStreamSynchronize(plan->last_stream) != cudaSuccess) return VSA_ERR_CUDA;
   int err = 0;
   int* dev_err = reinterpret_cast<int*>(plan->ws + plan->lay.err);
@@ -476,6 +596,7 @@ void vsa_plan_destroy(vsa_plan_t plan) {
   if (!plan) return;
   if (plan->ev[0])
     for (int i = 0; i < 4; ++i) cudaEventDestroy(plan->ev[i]);
+  host_path_free(plan->host);
   delete plan;
 }
 

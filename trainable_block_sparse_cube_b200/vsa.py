@@ -21,7 +21,7 @@ STATUS = {0: "VSA_OK", 1: "VSA_ERR_INVALID_ARG", 2: "VSA_ERR_SHAPE", 3: "VSA_ERR
 EXPORTED = ["vsa_workspace_bytes", "vsa_workspace_layout", "vsa_plan", "vsa_run", "vsa_run_fixed_idx",
             "vsa_forward", "vsa_check", "vsa_plan_destroy", "vsa_status_string", "vsa_set_wait_limit_ns",
             "vsa_set_debug_stall", "vsa_set_stage_timing", "vsa_stage_times", "vsa_kernels_per_run",
-            "vsa_forward_noalloc", "vsa_set_cube_major_copies"]
+            "vsa_forward_noalloc", "vsa_set_cube_major_copies", "vsa_run_host"]
 
 
 class VSAError(RuntimeError):
@@ -63,6 +63,8 @@ def load():
     L.vsa_run.argtypes = [vp] * 10
     L.vsa_run.restype = i32
     L.vsa_run_fixed_idx.argtypes = [vp] * 12
+    L.vsa_run_host.argtypes = [vp] * 10
+    L.vsa_run_host.restype = i32
     L.vsa_run_fixed_idx.restype = i32
     L.vsa_forward.argtypes = [vp] * 5 + [i32] * 7 + [ctypes.c_float, vp, vp, vp]
     L.vsa_forward.restype = i32
@@ -172,6 +174,25 @@ class Plan:
         cnt = torch.empty((self.B, self.heads, self.C), dtype=torch.int32, device=dev) if cnt is None else cnt
         _check(load().vsa_run(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(gate_c), _ptr(gate_f), _ptr(out), _ptr(idx),
                               _ptr(cnt), _stream()), "vsa_run")
+        return out, idx, cnt
+
+    def run_host(self, q, k, v, gate_c, gate_f, out, idx, cnt=None):
+        """Forward pass on host tensors (pinned for overlapped copies): inputs are
+        copied in and out/idx/cnt written back by the library; enqueued on the
+        current stream (synchronise it before reading the results)."""
+        BHND = (self.B, self.heads, self.N, self.D)
+        for t, n, dt, sh in ((q, "q", torch.bfloat16, BHND), (k, "k", torch.bfloat16, BHND),
+                             (v, "v", torch.bfloat16, BHND), (gate_c, "gate_c", torch.float32, BHND[:3]),
+                             (gate_f, "gate_f", torch.float32, BHND[:3]), (out, "out", torch.bfloat16, BHND),
+                             (idx, "idx", torch.int32, (self.B, self.heads, self.C, self.kcap)),
+                             (cnt, "cnt", torch.int32, (self.B, self.heads, self.C))):
+            if t is None and n == "cnt":
+                continue
+            if not isinstance(t, torch.Tensor) or t.is_cuda or t.dtype != dt or tuple(t.shape) != tuple(sh) \
+                    or not t.is_contiguous():
+                raise ValueError(f"{n} must be a contiguous host tensor of {dt} and shape {tuple(sh)}")
+        _check(load().vsa_run_host(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(gate_c), _ptr(gate_f), _ptr(out),
+                                   _ptr(idx), _ptr(cnt), _stream()), "vsa_run_host")
         return out, idx, cnt
 
     def run_fixed_idx(self, q, k, v, gate_c, gate_f, idx, cnt=None, want_out=True, want_coarse=False,
