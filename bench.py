@@ -31,7 +31,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from trainable_block_sparse_cube_b200 import synth  # noqa: E402
+from trainable_block_sparse_cube_b200 import replicas, synth  # noqa: E402
 
 METRIC = "VSA fwd ms/call & sparse TFLOP/s (% bf16 TC peak) at 61,440 tokens, K=32"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
@@ -230,16 +230,8 @@ def main():
     from trainable_block_sparse_cube_b200 import vsa
 
     torch.cuda.set_device(local)
-    dist = None
-    if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-
-    def barrier():
-        if dist is not None:
-            dist.barrier()
+    rep = replicas.from_env("nccl")
+    barrier = rep.barrier
 
     q, k, v, gc, gf = synth.make_inputs(wl)
     dq, dk, dv, dgc, dgf = (t.cuda() for t in (q, k, v, gc, gf))
@@ -280,14 +272,9 @@ def main():
     n_stage = len(range(0, args.steps, 10)) + (0 if (args.steps - 1) % 10 == 0 else 1)
     stage_ms = stage / n_stage
     plan.check()
-    total_ms = float(sum(step_ms))
-    t_max = total_ms
-    if dist is not None:
-        t = torch.tensor([total_ms], device=dq.device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_max = float(t.item())
+    t_max = rep.max_over_ranks(float(sum(step_ms)))
     ms_per_step = t_max / args.steps
-    value = world * (f_fine + f_coarse) * args.steps / (t_max * 1e-3) / 1e12
+    value = rep.job_throughput((f_fine + f_coarse) * args.steps, t_max * 1e-3) / 1e12
 
     # e2e through the C ABI's host-buffer entry point (vsa_run_host): pinned host
     # inputs -> device, forward, output + index lists -> host, all timed; the
@@ -306,12 +293,8 @@ def main():
         b.synchronize()
         if i >= 2:
             e2e_ms.append(a.elapsed_time(b))
-    e2e_t = sum(e2e_ms) if e2e_ms else float("nan")
-    if dist is not None:
-        t = torch.tensor([e2e_t], device=dq.device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_t = float(t.item())
-    e2e_val = world * (f_fine + f_coarse) * len(e2e_ms) / (e2e_t * 1e-3) / 1e12 if e2e_ms else None
+    e2e_t = rep.max_over_ranks(sum(e2e_ms) if e2e_ms else float("nan"))
+    e2e_val = rep.job_throughput((f_fine + f_coarse) * len(e2e_ms), e2e_t * 1e-3) / 1e12 if e2e_ms else None
     plan.check()
 
     peaks, peak_src = load_peaks()
@@ -346,10 +329,9 @@ def main():
         f, el, desc = oracle_sample(wl, args.cpu_seconds, q[0, 0], k[0, 0], v[0, 0], gc[0, 0], gf[0, 0])
         line["cpu_baseline"] = {"value": f / el / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
                                 "sample": f"{desc}; {el:.1f} s fp64 numpy"}
-    if rank == 0:
+    if rep.is_reporter:
         print(json.dumps(line), flush=True)
-    if dist is not None:
-        dist.destroy_process_group()
+    rep.close()
 
 
 if __name__ == "__main__":
