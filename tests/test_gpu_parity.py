@@ -29,6 +29,7 @@ SMALL = [
     W["pretrain16k"].with_(name="d64_k7", D=64, heads=2, T=8, H=8, W=24, topk=7),
     W["pretrain16k"].with_(name="k_eq_c", heads=1, T=4, H=8, W=12, topk=6),
     W["tiny"].with_(name="single_cube", T=4, H=4, W=4, heads=2, topk=1),
+    W["large77k"].with_(name="sin_k40_c80", heads=2, T=8, H=16, W=40, topk=40),
 ]
 
 

@@ -176,15 +176,17 @@ __device__ __forceinline__ void topk_from_candidates(const uint32_t* ckey, const
   }
 }
 
-// Fixed top-K <= 32 with the row's keys in shared memory instead of
+// Fixed top-K (any K), and the probabilities alone when the selection is
+// supplied by the caller, with the row's keys in shared memory instead of
 // registers, so more warps (rows) per SM hide the latency of the warp-wide
 // reductions. One warp per row; per warp the shared memory holds the keys
 // (C rounded up to 32) and kCandCap candidate ids. Passes: load the scores as
 // keys (lane maxima of score and key), the row sum, the probabilities as three
-// bf16 terms, then the selection through the candidates at or above the
-// lane-maxima bound, compacted in place; more than kCandCap candidates fall
-// back to the bit search over all keys.
-__global__ void __launch_bounds__(256, 4) coarse_select_small_kernel(const CoarseParams p) {
+// bf16 terms, then the selection. For K <= 32 the minimum of the lanes'
+// maxima bounds the K-th largest key from below, and the search runs over the
+// candidates at or above it, compacted in place; larger K, or more than
+// kCandCap candidates, take the bit search over all keys.
+__global__ void __launch_bounds__(256, 4) coarse_select_topk_kernel(const CoarseParams p) {
   extern __shared__ __align__(16) uint8_t dyn[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * 8 + warp;
@@ -237,13 +239,16 @@ __global__ void __launch_bounds__(256, 4) coarse_select_small_kernel(const Coars
   }
   if (!p.do_select) return;
   int32_t* irow = p.idx + (size_t)row * p.kcap;
-  // Lower bound lo of the Kt-th largest key (Kt <= 32 and every lane with a key
-  // holds one at or above it) and the row maximum hi.
+  // Lower bound lo of the Kt-th largest key (for Kt <= 32: every lane with a
+  // key holds one at or above it) and the row maximum hi.
   const uint32_t lo = __reduce_min_sync(0xffffffffu, lane < C ? lkmax : 0xffffffffu);
   const uint32_t hi = __reduce_max_sync(0xffffffffu, lkmax);
-  unsigned nl = 0;
-  for (int j = lane; j < C; j += 32) nl += (keys[j] >= lo);
-  const int n = (int)__reduce_add_sync(0xffffffffu, nl);
+  int n = kCandCap + 1;
+  if (Kt <= 32) {
+    unsigned nl = 0;
+    for (int j = lane; j < C; j += 32) nl += (keys[j] >= lo);
+    n = (int)__reduce_add_sync(0xffffffffu, nl);
+  }
   if (n <= kCandCap) {
     // In-place compaction in ascending id order: a candidate never lands past
     // the position it is read from, and every lane reads before the ballot.
@@ -294,10 +299,11 @@ __global__ void __launch_bounds__(256, 4) coarse_select_small_kernel(const Coars
   if (lane == 0) p.cnt[row] = Kt;
 }
 
-// Register-resident selection for top-K > 32 and top-p (TOPK: fixed top-K,
-// no top-p scratch, fewer registers).
-template <int PER, bool TOPK>
-__global__ void __launch_bounds__(256, TOPK ? 3 : 1) coarse_select_kernel(const CoarseParams p) {
+// Top-p selection, register-resident: the kmax best candidates (exact kmax-th
+// largest key, ties to the lower id) are ranked by score and cut at the first
+// prefix whose probability mass reaches top_p * l, clamped to [kmin, kmax].
+template <int PER>
+__global__ void __launch_bounds__(256, 1) coarse_select_topp_kernel(const CoarseParams p) {
   extern __shared__ __align__(16) uint8_t dyn[];
   __shared__ uint32_t cand_all[8][kCandCap];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -325,7 +331,7 @@ __global__ void __launch_bounds__(256, TOPK ? 3 : 1) coarse_select_kernel(const 
   l = warp_sum(l);
 
   if (p.do_select) {
-    const int Kt = p.topk > 0 ? p.topk : p.kmax;
+    const int Kt = p.kmax;
     // T is the Kt-th largest key exactly.
     const uint32_t T = kth_largest<PER>(key, C, Kt, cand_all[warp]);
     unsigned gtl = 0;
@@ -335,21 +341,7 @@ __global__ void __launch_bounds__(256, TOPK ? 3 : 1) coarse_select_kernel(const 
 
     int32_t* irow = p.idx + (size_t)row * p.kcap;
     int n_out;
-    if (TOPK) {
-      int pos = 0, eq_seen = 0;
-#pragma unroll
-      for (int u = 0; u < PER; ++u) {
-        const int j = lane + 32 * u;
-        const bool is_eq = (key[u] == T) && (j < C);
-        const unsigned eqb = __ballot_sync(0xffffffffu, is_eq);
-        const bool take = (key[u] > T) || (is_eq && eq_seen + __popc(eqb & lt_mask) < need);
-        const unsigned tb = __ballot_sync(0xffffffffu, take);
-        if (take) irow[pos + __popc(tb & lt_mask)] = j;
-        pos += __popc(tb);
-        eq_seen += __popc(eqb);
-      }
-      n_out = Kt;
-    } else {
+    {
       const int kmax = p.kmax;
       TopPScratch sc;
       uint8_t* base = dyn + (size_t)warp * kmax * 16;
@@ -602,30 +594,28 @@ cudaError_t launch_tc(const CoarseParams& p, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-template <int PER>
-cudaError_t launch_select(const CoarseParams& p, cudaStream_t st) {
+cudaError_t launch_select_topk(const CoarseParams& p, cudaStream_t st) {
   const int rows = p.BH * p.C;
-  if (p.topk > 0 && p.topk <= 32) {
-    const size_t smem = (size_t)8 * ((p.C + 31) / 32 * 32 + kCandCap) * 4;
-    if (smem > 48 * 1024) {
-      cudaError_t e = cudaFuncSetAttribute(coarse_select_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)smem);
-      if (e != cudaSuccess) return e;
-    }
-    coarse_select_small_kernel<<<(rows + 7) / 8, 256, smem, st>>>(p);
-    return cudaGetLastError();
-  }
-  if (!p.do_select || p.topk > 0) {
-    coarse_select_kernel<PER, true><<<(rows + 7) / 8, 256, 0, st>>>(p);
-    return cudaGetLastError();
-  }
-  const size_t smem = (size_t)8 * p.kmax * 16;
+  const size_t smem = (size_t)8 * ((p.C + 31) / 32 * 32 + kCandCap) * 4;
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(coarse_select_kernel<PER, false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(coarse_select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
     if (e != cudaSuccess) return e;
   }
-  coarse_select_kernel<PER, false><<<(rows + 7) / 8, 256, smem, st>>>(p);
+  coarse_select_topk_kernel<<<(rows + 7) / 8, 256, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <int PER>
+cudaError_t launch_select_topp(const CoarseParams& p, cudaStream_t st) {
+  const int rows = p.BH * p.C;
+  const size_t smem = (size_t)8 * p.kmax * 16;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(coarse_select_topp_kernel<PER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  coarse_select_topp_kernel<PER><<<(rows + 7) / 8, 256, smem, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -635,18 +625,19 @@ cudaError_t launch_coarse(const CoarseParams& p, cudaStream_t st) {
   cudaError_t e = p.D == 128 ? launch_tc<0, 128>(p, st) : launch_tc<0, 64>(p, st);
   if (e != cudaSuccess) return e;
   const int per = (p.C + 31) / 32;
-  if (per <= 1) e = launch_select<1>(p, st);
-  else if (per <= 2) e = launch_select<2>(p, st);
-  else if (per <= 4) e = launch_select<4>(p, st);
-  else if (per <= 8) e = launch_select<8>(p, st);
-  else if (per <= 16) e = launch_select<16>(p, st);
-  else if (per <= 24) e = launch_select<24>(p, st);
-  else if (per <= 32) e = launch_select<32>(p, st);
-  else if (per <= 40) e = launch_select<40>(p, st);
-  else if (per <= 48) e = launch_select<48>(p, st);
-  else if (per <= 64) e = launch_select<64>(p, st);
-  else if (per <= 96) e = launch_select<96>(p, st);
-  else e = launch_select<128>(p, st);
+  if (p.topk > 0 || !p.do_select) e = launch_select_topk(p, st);
+  else if (per <= 1) e = launch_select_topp<1>(p, st);
+  else if (per <= 2) e = launch_select_topp<2>(p, st);
+  else if (per <= 4) e = launch_select_topp<4>(p, st);
+  else if (per <= 8) e = launch_select_topp<8>(p, st);
+  else if (per <= 16) e = launch_select_topp<16>(p, st);
+  else if (per <= 24) e = launch_select_topp<24>(p, st);
+  else if (per <= 32) e = launch_select_topp<32>(p, st);
+  else if (per <= 40) e = launch_select_topp<40>(p, st);
+  else if (per <= 48) e = launch_select_topp<48>(p, st);
+  else if (per <= 64) e = launch_select_topp<64>(p, st);
+  else if (per <= 96) e = launch_select_topp<96>(p, st);
+  else e = launch_select_topp<128>(p, st);
   if (e != cudaSuccess) return e;
   return p.D == 128 ? launch_tc<1, 128>(p, st) : launch_tc<1, 64>(p, st);
 }
