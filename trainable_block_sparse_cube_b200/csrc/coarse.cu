@@ -58,74 +58,66 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// Per-warp scratch for top-p ranking: kmax entries of (id, key, weight) and
-// the weights in rank order.
-struct TopPScratch {
-  int* id;
-  uint32_t* key;
-  float* w;
-  float* sorted;
-};
-
-// Exact Kt-th largest key of the warp's row: the largest T with
-// #{key >= T} >= Kt, by an MSB-first search over the 32 key bits. For
-// Kt <= 32 the minimum of the lanes' maxima is a lower bound of the answer
-// (the 32 lane maxima are Kt or more keys at or above it), so the search runs
-// over the few keys at or above that bound, compacted into `cand` (kCandCap
-// per warp); it falls back to all keys when there are too many of them.
 constexpr int kCandCap = 256;
-template <int PER>
-__device__ __forceinline__ uint32_t kth_largest(const uint32_t (&key)[PER], int C, int Kt, uint32_t* cand) {
-  const int lane = threadIdx.x & 31;
-  const uint32_t lt_mask = (1u << lane) - 1u;
-  if (Kt <= 32) {
-    uint32_t lmax = 0;
-    bool any = false;
-#pragma unroll
-    for (int u = 0; u < PER; ++u)
-      if (lane + 32 * u < C) {
-        lmax = max(lmax, key[u]);
-        any = true;
-      }
-    const uint32_t lo = __reduce_min_sync(0xffffffffu, any ? lmax : 0xffffffffu);
-    unsigned nl = 0;
-#pragma unroll
-    for (int u = 0; u < PER; ++u) nl += (key[u] >= lo);
-    const int n = (int)__reduce_add_sync(0xffffffffu, nl);
-    if (n <= kCandCap) {
-      int pos = 0;
-#pragma unroll
-      for (int u = 0; u < PER; ++u) {
-        const bool t = key[u] >= lo;
-        const unsigned tb = __ballot_sync(0xffffffffu, t);
-        if (t) cand[pos + __popc(tb & lt_mask)] = key[u];
-        pos += __popc(tb);
-      }
-      __syncwarp();
-      uint32_t ck[kCandCap / 32];
-#pragma unroll
-      for (int i = 0; i < kCandCap / 32; ++i) ck[i] = (lane + 32 * i < n) ? cand[lane + 32 * i] : 0u;
-      __syncwarp();
-      uint32_t T = 0;
-      for (int b = 31; b >= 0; --b) {
-        const uint32_t c = T | (1u << b);
-        unsigned cnt = 0;
-#pragma unroll
-        for (int i = 0; i < kCandCap / 32; ++i) cnt += (ck[i] >= c);
-        if ((int)__reduce_add_sync(0xffffffffu, cnt) >= Kt) T = c;
-      }
-      return T;
-    }
-  }
+
+// MSB-first search for the Kt-th largest of the row's C keys (in shared
+// memory): the largest T with #{key >= T} >= Kt.
+__device__ __forceinline__ uint32_t kth_largest(const uint32_t* keys, int C, int Kt, int lane) {
   uint32_t T = 0;
   for (int b = 31; b >= 0; --b) {
     const uint32_t c = T | (1u << b);
     unsigned cnt = 0;
-#pragma unroll
-    for (int u = 0; u < PER; ++u) cnt += (key[u] >= c);
+    for (int j = lane; j < C; j += 32) cnt += (keys[j] >= c);
     if ((int)__reduce_add_sync(0xffffffffu, cnt) >= Kt) T = c;
   }
   return T;
+}
+
+// Loads row `row` of the scores into shared memory as order-preserving keys,
+// then writes its softmax probabilities as three bf16 terms (zero in the
+// padding columns C .. Cp-1), the A operand of the output product. Returns
+// the row max in log2 units (mb), the row sum l and this lane's largest key.
+__device__ __forceinline__ void row_softmax(const CoarseParams& p, int row, uint32_t* keys, int lane, float& mb,
+                                            float& l, uint32_t& lkmax) {
+  const int C = p.C;
+  const float* srow = p.s + (size_t)row * C;
+  float lm = -INFINITY;
+  lkmax = 0;
+  for (int j0 = 0; j0 < C; j0 += 256) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = j0 + lane + 32 * u;
+      v[u] = j < C ? srow[j] : -INFINITY;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = j0 + lane + 32 * u;
+      if (j < C) {
+        const uint32_t k = order_key(v[u]);
+        keys[j] = k;
+        lkmax = max(lkmax, k);
+        lm = fmaxf(lm, v[u]);
+      }
+    }
+  }
+  mb = warp_max(lm) * kLog2e;
+  __syncwarp();
+  float ls = 0.f;
+  for (int j = lane; j < C; j += 32) ls += fast_exp2(fmaf(key_value(keys[j]), kLog2e, -mb));
+  l = warp_sum(ls);
+  const float inv_l = 1.0f / l;
+  const size_t plane = (size_t)p.BH * C * p.Cp;
+  __nv_bfloat16* prow = p.psplit + (size_t)row * p.Cp;
+  for (int j = lane; j < p.Cp; j += 32) {
+    const float x = j < C ? fast_exp2(fmaf(key_value(keys[j]), kLog2e, -mb)) * inv_l : 0.f;
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    const float r1 = x - __bfloat162float(h);
+    const __nv_bfloat16 md = __float2bfloat16_rn(r1);
+    prow[j] = h;
+    prow[plane + j] = md;
+    prow[2 * plane + j] = __float2bfloat16_rn(r1 - __bfloat162float(md));
+  }
 }
 
 // Top-K emission for Kt <= 32 from the candidates (keys at or above the lower
@@ -195,48 +187,10 @@ __global__ void __launch_bounds__(256, 4) coarse_select_topk_kernel(const Coarse
   const int stride = (C + 31) / 32 * 32;
   uint32_t* keys = reinterpret_cast<uint32_t*>(dyn) + (size_t)warp * (stride + kCandCap);
   int* cidx = reinterpret_cast<int*>(keys + stride);
-  const float* srow = p.s + (size_t)row * C;
   const uint32_t lt_mask = (1u << lane) - 1u;
-
-  float lm = -INFINITY;
-  uint32_t lkmax = 0;
-  for (int j0 = 0; j0 < C; j0 += 256) {
-    float v[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int j = j0 + lane + 32 * u;
-      v[u] = j < C ? srow[j] : -INFINITY;
-    }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int j = j0 + lane + 32 * u;
-      if (j < C) {
-        const uint32_t k = order_key(v[u]);
-        keys[j] = k;
-        lkmax = max(lkmax, k);
-        lm = fmaxf(lm, v[u]);
-      }
-    }
-  }
-  const float m = warp_max(lm);
-  const float mb = m * kLog2e;
-  __syncwarp();
-  float l = 0.f;
-  for (int j = lane; j < C; j += 32) l += fast_exp2(fmaf(key_value(keys[j]), kLog2e, -mb));
-  l = warp_sum(l);
-  // Probabilities as three bf16 terms (zero in the padding columns C .. Cp-1).
-  const float inv_l = 1.0f / l;
-  const size_t plane = (size_t)p.BH * C * p.Cp;
-  __nv_bfloat16* prow = p.psplit + (size_t)row * p.Cp;
-  for (int j = lane; j < p.Cp; j += 32) {
-    const float x = j < C ? fast_exp2(fmaf(key_value(keys[j]), kLog2e, -mb)) * inv_l : 0.f;
-    const __nv_bfloat16 h = __float2bfloat16_rn(x);
-    const float r1 = x - __bfloat162float(h);
-    const __nv_bfloat16 md = __float2bfloat16_rn(r1);
-    prow[j] = h;
-    prow[plane + j] = md;
-    prow[2 * plane + j] = __float2bfloat16_rn(r1 - __bfloat162float(md));
-  }
+  float mb, l;
+  uint32_t lkmax;
+  row_softmax(p, row, keys, lane, mb, l, lkmax);
   if (!p.do_select) return;
   int32_t* irow = p.idx + (size_t)row * p.kcap;
   // Lower bound lo of the Kt-th largest key (for Kt <= 32: every lane with a
@@ -273,13 +227,7 @@ __global__ void __launch_bounds__(256, 4) coarse_select_topk_kernel(const Coarse
   } else {
     // Bit search for the Kt-th largest key over all keys, then the ids above it
     // and the lowest-id ones equal to it, ascending.
-    uint32_t T = 0;
-    for (int b = 31; b >= 0; --b) {
-      const uint32_t c = T | (1u << b);
-      unsigned cnt = 0;
-      for (int j = lane; j < C; j += 32) cnt += (keys[j] >= c);
-      if ((int)__reduce_add_sync(0xffffffffu, cnt) >= Kt) T = c;
-    }
+    const uint32_t T = kth_largest(keys, C, Kt, lane);
     unsigned gt = 0;
     for (int j = lane; j < C; j += 32) gt += (keys[j] > T);
     const int need = Kt - (int)__reduce_add_sync(0xffffffffu, gt);
@@ -299,141 +247,104 @@ __global__ void __launch_bounds__(256, 4) coarse_select_topk_kernel(const Coarse
   if (lane == 0) p.cnt[row] = Kt;
 }
 
-// Top-p selection, register-resident: the kmax best candidates (exact kmax-th
-// largest key, ties to the lower id) are ranked by score and cut at the first
-// prefix whose probability mass reaches top_p * l, clamped to [kmin, kmax].
-template <int PER>
-__global__ void __launch_bounds__(256, 1) coarse_select_topp_kernel(const CoarseParams p) {
+// Top-p selection with the row's keys in shared memory: the kmax best
+// candidates (the exact kmax-th largest key by the bit search, ties to the
+// lower id) are ranked by score and cut at the first prefix whose probability
+// mass reaches top_p * l, clamped to [kmin, kmax]; the ids go out ascending.
+// One warp per row; per warp the shared memory holds the keys (C rounded up
+// to 32) and four kmax-entry arrays: candidate id (with its rank packed above
+// it), key, weight, and the weights in rank order. Warps per CTA: blockDim / 32.
+__global__ void __launch_bounds__(256, 2) coarse_select_topp_kernel(const CoarseParams p) {
   extern __shared__ __align__(16) uint8_t dyn[];
-  __shared__ uint32_t cand_all[8][kCandCap];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * 8 + warp;
+  const int row = blockIdx.x * (blockDim.x >> 5) + warp;
   if (row >= p.BH * p.C) return;
-  const int C = p.C;
-  float* srow = p.s + (size_t)row * C;
+  const int C = p.C, Kt = p.kmax;
+  const int stride = (C + 31) / 32 * 32;
+  uint32_t* keys = reinterpret_cast<uint32_t*>(dyn) + (size_t)warp * (stride + 4 * Kt);
+  int* cid = reinterpret_cast<int*>(keys + stride);
+  uint32_t* ckey = keys + stride + Kt;
+  float* cw = reinterpret_cast<float*>(keys + stride + 2 * Kt);
+  float* sorted = reinterpret_cast<float*>(keys + stride + 3 * Kt);
   const uint32_t lt_mask = (1u << lane) - 1u;
+  float mb, l;
+  uint32_t lkmax;
+  row_softmax(p, row, keys, lane, mb, l, lkmax);
+  int32_t* irow = p.idx + (size_t)row * p.kcap;
 
-  uint32_t key[PER];
-  float m = -INFINITY;
-#pragma unroll
-  for (int u = 0; u < PER; ++u) {
-    const int j = lane + 32 * u;
-    const float s = (j < C) ? srow[j] : -INFINITY;
-    key[u] = (j < C) ? order_key(s) : 0u;
-    m = fmaxf(m, s);
-  }
-  m = warp_max(m);
-  const float mb = m * kLog2e;
-  float l = 0.f;
-#pragma unroll
-  for (int u = 0; u < PER; ++u)
-    if (lane + 32 * u < C) l += fast_exp2(fmaf(key_value(key[u]), kLog2e, -mb));
-  l = warp_sum(l);
-
-  if (p.do_select) {
-    const int Kt = p.kmax;
-    // T is the Kt-th largest key exactly.
-    const uint32_t T = kth_largest<PER>(key, C, Kt, cand_all[warp]);
-    unsigned gtl = 0;
-#pragma unroll
-    for (int u = 0; u < PER; ++u) gtl += (key[u] > T);
-    const int need = Kt - (int)__reduce_add_sync(0xffffffffu, gtl);  // ids equal to T to take, lowest first
-
-    int32_t* irow = p.idx + (size_t)row * p.kcap;
-    int n_out;
-    {
-      const int kmax = p.kmax;
-      TopPScratch sc;
-      uint8_t* base = dyn + (size_t)warp * kmax * 16;
-      sc.id = reinterpret_cast<int*>(base);
-      sc.key = reinterpret_cast<uint32_t*>(base + kmax * 4);
-      sc.w = reinterpret_cast<float*>(base + kmax * 8);
-      sc.sorted = reinterpret_cast<float*>(base + kmax * 12);
-      int pos = 0, eq_seen = 0;
-#pragma unroll
-      for (int u = 0; u < PER; ++u) {
-        const int j = lane + 32 * u;
-        const bool is_eq = (key[u] == T) && (j < C);
-        const unsigned eqb = __ballot_sync(0xffffffffu, is_eq);
-        const bool take = (key[u] > T) || (is_eq && eq_seen + __popc(eqb & lt_mask) < need);
-        const unsigned tb = __ballot_sync(0xffffffffu, take);
-        if (take) {
-          const int q = pos + __popc(tb & lt_mask);
-          sc.id[q] = j;
-          sc.key[q] = key[u];
-          sc.w[q] = fast_exp2(fmaf(key_value(key[u]), kLog2e, -mb));
-        }
-        pos += __popc(tb);
-        eq_seen += __popc(eqb);
-      }
-      __syncwarp();
-      // Rank = number of candidates ahead in (score desc, id asc) order.
-      for (int c = lane; c < Kt; c += 32) {
-        const uint32_t kc = sc.key[c];
-        int r = 0;
-        for (int o = 0; o < Kt; ++o) {
-          const uint32_t ko = sc.key[o];
-          r += (ko > kc) || (ko == kc && o < c);  // candidates are stored in ascending id
-        }
-        sc.sorted[r] = sc.w[c];
-        sc.id[c] = sc.id[c] | (r << 16);  // pack rank above the id (ids < 65536)
-      }
-      __syncwarp();
-      // First rank whose cumulative weight reaches top_p * l.
-      const int CH = (Kt + 31) / 32;
-      const int b0 = lane * CH, b1 = min(b0 + CH, Kt);
-      float part = 0.f;
-      for (int r = b0; r < b1; ++r) part += sc.sorted[r];
-      float incl = part;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const float y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      float run = incl - part;
-      const float target = p.top_p * l;
-      int first = 0x7fffffff;
-      for (int r = b0; r < b1; ++r) {
-        run += sc.sorted[r];
-        if (run >= target) { first = r; break; }
-      }
-      first = __reduce_min_sync(0xffffffffu, first);
-      int nsel = (first == 0x7fffffff) ? Kt : first + 1;
-      nsel = max(nsel, p.kmin);
-      nsel = min(nsel, Kt);
-      // Emit candidates with rank < nsel in ascending id order.
-      int opos = 0;
-      for (int c0 = 0; c0 < Kt; c0 += 32) {
-        const int c = c0 + lane;
-        int packed = (c < Kt) ? sc.id[c] : 0;
-        const bool take = (c < Kt) && ((packed >> 16) < nsel);
-        const unsigned tb = __ballot_sync(0xffffffffu, take);
-        if (take) irow[opos + __popc(tb & lt_mask)] = packed & 0xffff;
-        opos += __popc(tb);
-      }
-      n_out = nsel;
+  // The Kt candidates: keys above the Kt-th largest T and the lowest-id ones
+  // equal to it, in ascending id order, with their softmax numerators.
+  const uint32_t T = kth_largest(keys, C, Kt, lane);
+  unsigned gtl = 0;
+  for (int j = lane; j < C; j += 32) gtl += (keys[j] > T);
+  const int need = Kt - (int)__reduce_add_sync(0xffffffffu, gtl);
+  int pos = 0, eq_seen = 0;
+  for (int j0 = 0; j0 < C; j0 += 32) {
+    const int j = j0 + lane;
+    const uint32_t k = j < C ? keys[j] : 0u;
+    const bool is_eq = j < C && k == T;
+    const unsigned eqb = __ballot_sync(0xffffffffu, is_eq);
+    const bool take = (j < C && k > T) || (is_eq && eq_seen + __popc(eqb & lt_mask) < need);
+    const unsigned tb = __ballot_sync(0xffffffffu, take);
+    if (take) {
+      const int q = pos + __popc(tb & lt_mask);
+      cid[q] = j;
+      ckey[q] = k;
+      cw[q] = fast_exp2(fmaf(key_value(k), kLog2e, -mb));
     }
-    for (int c = n_out + lane; c < p.kcap; c += 32) irow[c] = -1;
-    if (lane == 0) p.cnt[row] = n_out;
+    pos += __popc(tb);
+    eq_seen += __popc(eqb);
   }
-  // Probabilities over the scores as three bf16 terms (zero in the padding
-  // columns C .. Cp-1), the A operand of the output product.
-  const float inv_l = 1.0f / l;
-  const size_t plane = (size_t)p.BH * C * p.Cp;
-  __nv_bfloat16* prow = p.psplit + (size_t)row * p.Cp;
+  __syncwarp();
+  // Rank = number of candidates ahead in (score desc, id asc) order.
+  for (int c = lane; c < Kt; c += 32) {
+    const uint32_t kc = ckey[c];
+    int r = 0;
+    for (int o = 0; o < Kt; ++o) {
+      const uint32_t ko = ckey[o];
+      r += (ko > kc) || (ko == kc && o < c);  // candidates are stored in ascending id
+    }
+    sorted[r] = cw[c];
+    cid[c] = cid[c] | (r << 16);  // pack rank above the id (ids < 65536)
+  }
+  __syncwarp();
+  // First rank whose cumulative weight reaches top_p * l.
+  const int CH = (Kt + 31) / 32;
+  const int b0 = lane * CH, b1 = min(b0 + CH, Kt);
+  float part = 0.f;
+  for (int r = b0; r < b1; ++r) part += sorted[r];
+  float incl = part;
 #pragma unroll
-  for (int u = 0; u < PER; ++u) {
-    const int j = lane + 32 * u;
-    if (j < p.Cp) {
-      const float x = j < C ? fast_exp2(fmaf(key_value(key[u]), kLog2e, -mb)) * inv_l : 0.f;
-      const __nv_bfloat16 h = __float2bfloat16_rn(x);
-      const float r1 = x - __bfloat162float(h);
-      const __nv_bfloat16 m = __float2bfloat16_rn(r1);
-      prow[j] = h;
-      prow[plane + j] = m;
-      prow[2 * plane + j] = __float2bfloat16_rn(r1 - __bfloat162float(m));
+  for (int o = 1; o < 32; o <<= 1) {
+    const float y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  float run = incl - part;
+  const float target = p.top_p * l;
+  int first = 0x7fffffff;
+  for (int r = b0; r < b1; ++r) {
+    run += sorted[r];
+    if (run >= target) {
+      first = r;
+      break;
     }
   }
+  first = __reduce_min_sync(0xffffffffu, first);
+  int nsel = (first == 0x7fffffff) ? Kt : first + 1;
+  nsel = max(nsel, p.kmin);
+  nsel = min(nsel, Kt);
+  // Candidates with rank < nsel, in ascending id order.
+  int opos = 0;
+  for (int c0 = 0; c0 < Kt; c0 += 32) {
+    const int c = c0 + lane;
+    const int packed = (c < Kt) ? cid[c] : 0;
+    const bool take = (c < Kt) && ((packed >> 16) < nsel);
+    const unsigned tb = __ballot_sync(0xffffffffu, take);
+    if (take) irow[opos + __popc(tb & lt_mask)] = packed & 0xffff;
+    opos += __popc(tb);
+  }
+  for (int c = nsel + lane; c < p.kcap; c += 32) irow[c] = -1;
+  if (lane == 0) p.cnt[row] = nsel;
 }
 
 // ------------------------------------------------------------ 1 / 3. three-term bf16 GEMM
@@ -606,16 +517,18 @@ cudaError_t launch_select_topk(const CoarseParams& p, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-template <int PER>
 cudaError_t launch_select_topp(const CoarseParams& p, cudaStream_t st) {
   const int rows = p.BH * p.C;
-  const size_t smem = (size_t)8 * p.kmax * 16;
+  const size_t per_warp = ((size_t)(p.C + 31) / 32 * 32 + 4 * (size_t)p.kmax) * 4;
+  int wpc = 8;  // warps (rows) per CTA, as many as fit in 227 KB of shared memory
+  while (wpc > 1 && per_warp * wpc > 227 * 1024) --wpc;
+  const size_t smem = per_warp * wpc;
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(coarse_select_topp_kernel<PER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(coarse_select_topp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
   }
-  coarse_select_topp_kernel<PER><<<(rows + 7) / 8, 256, smem, st>>>(p);
+  coarse_select_topp_kernel<<<(rows + wpc - 1) / wpc, 32 * wpc, smem, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -624,20 +537,7 @@ cudaError_t launch_select_topp(const CoarseParams& p, cudaStream_t st) {
 cudaError_t launch_coarse(const CoarseParams& p, cudaStream_t st) {
   cudaError_t e = p.D == 128 ? launch_tc<0, 128>(p, st) : launch_tc<0, 64>(p, st);
   if (e != cudaSuccess) return e;
-  const int per = (p.C + 31) / 32;
-  if (p.topk > 0 || !p.do_select) e = launch_select_topk(p, st);
-  else if (per <= 1) e = launch_select_topp<1>(p, st);
-  else if (per <= 2) e = launch_select_topp<2>(p, st);
-  else if (per <= 4) e = launch_select_topp<4>(p, st);
-  else if (per <= 8) e = launch_select_topp<8>(p, st);
-  else if (per <= 16) e = launch_select_topp<16>(p, st);
-  else if (per <= 24) e = launch_select_topp<24>(p, st);
-  else if (per <= 32) e = launch_select_topp<32>(p, st);
-  else if (per <= 40) e = launch_select_topp<40>(p, st);
-  else if (per <= 48) e = launch_select_topp<48>(p, st);
-  else if (per <= 64) e = launch_select_topp<64>(p, st);
-  else if (per <= 96) e = launch_select_topp<96>(p, st);
-  else e = launch_select_topp<128>(p, st);
+  e = (p.topk > 0 || !p.do_select) ? launch_select_topk(p, st) : launch_select_topp(p, st);
   if (e != cudaSuccess) return e;
   return p.D == 128 ? launch_tc<1, 128>(p, st) : launch_tc<1, 64>(p, st);
 }
