@@ -23,6 +23,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -93,8 +94,10 @@ class ClockSampler:
         self.path = None
 
     def start(self):
-        os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{self.gpu}.csv")
+        # raw samples go to VSA_BENCH_LOG_DIR (default: the temp directory)
+        log_dir = os.environ.get("VSA_BENCH_LOG_DIR") or tempfile.gettempdir()
+        os.makedirs(log_dir, exist_ok=True)
+        self.path = os.path.join(log_dir, f"clocks_gpu{self.gpu}.csv")
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu=timestamp,{self.FIELDS}",

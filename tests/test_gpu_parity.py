@@ -239,3 +239,31 @@ def test_host_buffers_match_device_run(wl):
         assert torch.equal(hout, out.cpu()) and torch.equal(hidx, idx.cpu()) and torch.equal(hcnt, cnt.cpu())
         hout.zero_()
         hidx.fill_(-5)
+
+
+@pytest.mark.parametrize("mode", ["topk_all", "topp_kmax1024"])
+def test_maximum_cube_count(mode):
+    """C = 4096 cubes, the largest the library accepts: every select kernel
+    holds a whole 4096-key row in shared memory. topk_all selects every cube
+    (K = C, the degenerate case where the fine stage is dense attention over
+    all 262,144 keys); topp_kmax1024 runs top-p with the largest kmax."""
+    if mode == "topk_all":
+        wl = W["pretrain16k"].with_(name="max_c_all", heads=1, D=64, T=16, H=64, W=256, topk=4096)
+    else:
+        wl = W["dynamic61k"].with_(name="max_c_topp", heads=1, D=64, T=16, H=64, W=256, kmin=4, kmax=1024)
+    assert wl.C == 4096
+    inputs = synth.make_inputs(wl)
+    q, k, v, gc, gf = inputs
+    plan, dev_in, out, idx, cnt = _run(wl, inputs)
+    idx_h, cnt_h = idx[0, 0].cpu().numpy(), cnt[0, 0].cpu().numpy()
+    if mode == "topk_all":
+        assert (cnt_h == 4096).all()
+        assert (idx_h == np.arange(4096, dtype=np.int32)[None, :]).all()
+    else:
+        rsel = oracle_head(wl, q, k, v, gc, gf, 0, 0, query_cubes=[])
+        check_lists(wl, rsel, idx_h, cnt_h)
+    cubes = [0, 1777, 4095]
+    r = oracle_head(wl, q, k, v, gc, gf, 0, 0, query_cubes=cubes, lists_in=idx_h, counts_in=cnt_h)
+    toks = np.concatenate([r["perm"][64 * c: 64 * c + 64] for c in cubes])
+    got = out[0, 0, torch.from_numpy(toks).cuda()].float().cpu().numpy()
+    assert_close(got, r["out"][toks], f"{mode} sampled output")
