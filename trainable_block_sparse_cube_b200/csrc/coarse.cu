@@ -349,7 +349,8 @@ __global__ void __launch_bounds__(256, 2) coarse_select_topp_kernel(const Coarse
 
 // ------------------------------------------------------------ 1 / 3. three-term bf16 GEMM
 // One CTA per 128-row tile: warp 0 issues the TMA loads (all three terms of A
-// and B for 64 columns of K per stage, two stages), warp 1 the 6 x 4 MMAs of
+// and B for 64 columns of K per stage; one stage for the scores, two for the
+// output), warp 1 the 6 x 4 MMAs of
 // a stage (M=128, K=16 each), and all four warps read the fp32 accumulator
 // out of tensor memory.
 //   KIND 0 (scores): A = qbar terms [C x D], B = kbar terms [C x D] (both
@@ -363,11 +364,15 @@ struct TcShape {
   static constexpr int A_BYTES = 128 * 64 * 2;      // one term, 128 rows x 64 K
   static constexpr int B_BYTES = NT * 64 * 2;       // one term
   static constexpr int STAGE = 3 * (A_BYTES + B_BYTES);
-  static constexpr int SMEM = 2 * STAGE + 1024;
+  // Scores: K = D is one or two 64-column chunks, so a single stage lets two
+  // CTAs share an SM and overlap each other's loads, MMAs and epilogue.
+  // Output: K = Cp is up to 64 chunks, double-buffered.
+  static constexpr int NS = KIND == 0 ? 1 : 2;
+  static constexpr int SMEM = NS * STAGE + 1024;
 };
 
 template <int KIND, int D>
-__global__ void __launch_bounds__(128, 1) coarse_tc_kernel(const __grid_constant__ CoarseParams p) {
+__global__ void __launch_bounds__(128, KIND == 0 ? 2 : 1) coarse_tc_kernel(const __grid_constant__ CoarseParams p) {
   using S = TcShape<KIND, D>;
   using namespace ptx;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -404,8 +409,8 @@ __global__ void __launch_bounds__(128, 1) coarse_tc_kernel(const __grid_constant
     const CUtensorMap* tb = KIND == 0 ? &p.tm_ks : &p.tm_vs;
     int armed = 0;
     for (int c = 0; c < nch; ++c) {
-      const int st = c & 1;
-      if (c >= 2 && !mbar_wait(&empty[st], ((c >> 1) - 1) & 1, lim)) {
+      const int st = c % S::NS;
+      if (c >= S::NS && !mbar_wait(&empty[st], ((c / S::NS) - 1) & 1, lim)) {
         atomicOr(p.err, kErrTimeout);
         break;
       }
@@ -422,15 +427,15 @@ __global__ void __launch_bounds__(128, 1) coarse_tc_kernel(const __grid_constant
       }
     }
     // Drain: the last armed phase of each stage covers all copies issued.
-    for (int st = 0; st < 2 && st < armed; ++st) mbar_wait(&full[st], (((armed - 1 - st) >> 1)) & 1, lim);
+    for (int st = 0; st < S::NS && st < armed; ++st) mbar_wait(&full[st], ((armed - 1 - st) / S::NS) & 1, lim);
   } else if (warp == 1 && lane == 0) {
     constexpr uint32_t idesc = idesc_bf16_f32(128, S::NT, false, KIND == 1);
     // Term pairs (A term, B term) of the six products kept.
     constexpr int pa[6] = {2, 0, 1, 1, 0, 0}, pb[6] = {0, 2, 1, 0, 1, 0};
     bool ok = true;
     for (int c = 0; c < nch && ok; ++c) {
-      const int st = c & 1;
-      if (!mbar_wait(&full[st], (c >> 1) & 1, lim)) {
+      const int st = c % S::NS;
+      if (!mbar_wait(&full[st], (c / S::NS) & 1, lim)) {
         atomicOr(p.err, kErrTimeout);
         ok = false;
         break;
