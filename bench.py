@@ -323,6 +323,12 @@ def main():
         "gather_pool_gbs": gather_bytes / (stage_ms[0] * 1e-3) / 1e9,
         "gather_pool_frac_hbm": gather_bytes / (stage_ms[0] * 1e-3) / 1e9 / hbm,
         "coarse_share": float(stage_ms[1]) / float(stage_ms.sum()),
+        # coarse stage: its FLOPs (two C x C x D products per head) and the bytes it
+        # must move (three-term means in, scores and three-term P written and read
+        # back, lists, coarse output), over its event-timed duration
+        "coarse_tflops": f_coarse / (stage_ms[1] * 1e-3) / 1e12,
+        "coarse_gbs": (9.0 * BH * C * D * 2 + 2.0 * BH * C * C * 4 + 2.0 * 3 * BH * C * ((C + 7) // 8 * 8) * 2
+                       + BH * C * wl.kcap * 4 + BH * C * D * 4) / (stage_ms[1] * 1e-3) / 1e9,
         "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_t / len(e2e_ms) if e2e_ms else None},
         "gpu_launches": vsa.load().vsa_kernels_per_run() * args.steps,
