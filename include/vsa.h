@@ -149,8 +149,10 @@ vsa_status vsa_run_host(vsa_plan_t plan, const void* q, const void* k, const voi
                         const float* gate_f, void* out, int32_t* idx, int32_t* cnt, void* stream);
 
 /* One-call form. Keeps a library-owned plan and workspace per distinct
- * configuration (the first call for a configuration allocates device memory
- * with cudaMalloc; later calls allocate nothing). topk > 0 selects top-K;
+ * configuration and device (the first call for a configuration allocates
+ * device memory with cudaMalloc; later calls allocate nothing). At most 16
+ * configurations are kept, for the life of the process; a call with a 17th
+ * returns VSA_ERR_UNSUPPORTED (use vsa_plan for more). topk > 0 selects top-K;
  * topk == 0 selects top-p with kmin = 4 and kmax = min(128, C). */
 vsa_status vsa_forward(const void* q, const void* k, const void* v, const float* gate_c, const float* gate_f,
                        int B, int heads, int T, int H, int W, int D, int topk, float top_p, void* out, int32_t* idx,
