@@ -34,7 +34,7 @@ import numpy as np
 
 __all__ = [
     "cube_perm", "pool_cubes", "coarse_attention", "select_topk", "select_topp",
-    "fine_attention", "gated_combine", "forward_head", "forward",
+    "fine_attention", "gated_combine", "forward_head",
 ]
 
 
@@ -222,28 +222,3 @@ def forward_head(q, k, v, gate_c, gate_f, T, H, W, topk=0, top_p=0.0, kmin=1, km
     out = gated_combine(Oc, Of, gate_c, gate_f, perm)
     return dict(perm=perm, qbar=qbar, kbar=kbar, vbar=vbar, s=s, P=P, Oc=Oc,
                 lists=lists, counts=counts, Of=Of, out=out)
-
-
-def forward(q, k, v, gate_c, gate_f, T, H, W, topk=0, top_p=0.0, kmin=1, kmax=None):
-    """Batched form over [B, heads, N, D]; loops over (b, head).
-
-    Returns (out [B,h,N,D], lists [B,h,C,Kcap] padded -1, counts [B,h,C],
-    Oc [B,h,C,D], Of [B,h,N,D], s [B,h,C,C])."""
-    q, k, v = (np.asarray(x) for x in (q, k, v))
-    B, nh, N, D = q.shape
-    C = N // 64
-    kcap = topk if topk > 0 else (C if kmax is None else kmax)
-    out = np.empty((B, nh, N, D))
-    Of = np.empty((B, nh, N, D))
-    Oc = np.empty((B, nh, C, D))
-    S = np.empty((B, nh, C, C))
-    lists = np.full((B, nh, C, kcap), -1, dtype=np.int64)
-    counts = np.empty((B, nh, C), dtype=np.int64)
-    for b in range(B):
-        for h in range(nh):
-            r = forward_head(q[b, h], k[b, h], v[b, h], gate_c[b, h], gate_f[b, h], T, H, W,
-                             topk, top_p, kmin, kmax)
-            out[b, h], Of[b, h], Oc[b, h], S[b, h] = r["out"], r["Of"], r["Oc"], r["s"]
-            lists[b, h, :, : r["lists"].shape[1]] = r["lists"]
-            counts[b, h] = r["counts"]
-    return out, lists, counts, Oc, Of, S

@@ -65,7 +65,9 @@ def test_small_all_stages(wl):
     BH = wl.B * wl.heads
     qc = plan.cube_major("q").cpu().view(wl.B, wl.heads, wl.C * 64, wl.D)
     vcm = plan.cube_major("v").cpu().view(wl.B, wl.heads, wl.C * 64, wl.D)
+    qpool = plan.pooled("q").cpu().view(wl.B, wl.heads, wl.C, wl.D)
     kpool = plan.pooled("k").cpu().view(wl.B, wl.heads, wl.C, wl.D)
+    vpool = plan.pooled("v").cpu().view(wl.B, wl.heads, wl.C, wl.D)
     idx_h, cnt_h, out_h = idx.cpu().numpy(), cnt.cpu().numpy(), out.float().cpu().numpy()
     ref_idx = np.zeros((wl.B, wl.heads, wl.C, wl.kcap), dtype=np.int32)
     ref_cnt = np.zeros((wl.B, wl.heads, wl.C), dtype=np.int32)
@@ -78,7 +80,9 @@ def test_small_all_stages(wl):
             r = oracle_head(wl, q, k, v, gc, gf, b, h)
             refs[b, h] = r
             # a2 pool
+            assert_close(qpool[b, h].numpy(), r["qbar"], "pooled q", max_abs=1e-5, mean_abs=1e-6)
             assert_close(kpool[b, h].numpy(), r["kbar"], "pooled k", max_abs=1e-5, mean_abs=1e-6)
+            assert_close(vpool[b, h].numpy(), r["vbar"], "pooled v", max_abs=1e-5, mean_abs=1e-6)
             # a4 selection
             check_lists(wl, r, idx_h[b, h], cnt_h[b, h])
             ref_idx[b, h], ref_cnt[b, h] = _padded(r["lists"], r["counts"], wl.kcap)
@@ -100,6 +104,14 @@ def test_small_all_stages(wl):
 
 @pytest.mark.parametrize("name", ["pretrain16k", "long61k_k32", "long61k_k16", "large77k", "dynamic61k"])
 def test_full_size_sampled(name):
+    """Full-size workloads, sampled heads.
+
+    Per sampled head: every selection row against the oracle's fp64 scores;
+    the whole pass on the GPU's own lists at sampled query cubes; then the
+    fixed-selection path on the oracle's own lists (the other heads keep the
+    GPU's lists), which at these sizes gives each CTA several items: the
+    coarse output of every cube, and the fine output before gating and the
+    gated output at the sampled cubes, element by element."""
     wl = W[name]
     inputs = synth.make_inputs(wl)
     q, k, v, gc, gf = inputs
@@ -107,6 +119,9 @@ def test_full_size_sampled(name):
     heads = sorted({0, wl.heads // 2, wl.heads - 1})
     rng = np.random.default_rng(11)
     exact = exempt = 0
+    idx_or = idx.clone()
+    cnt_or = cnt.clone()
+    sampled = {}
     for h in heads:
         idx_h = idx[0, h].cpu().numpy()
         cnt_h = cnt[0, h].cpu().numpy()
@@ -120,9 +135,20 @@ def test_full_size_sampled(name):
         toks = np.concatenate([r["perm"][64 * c: 64 * c + 64] for c in cubes])
         got = out[0, h, torch.from_numpy(toks).cuda()].float().cpu().numpy()
         assert_close(got, r["out"][toks], f"{name} head {h} sampled output")
-        # the same rows through the fixed-selection path with the oracle's lists
-        oc_ref = r["Oc"]
-        assert np.isfinite(oc_ref).all()
+        ref_idx, ref_cnt = _padded(rsel["lists"], rsel["counts"], wl.kcap)
+        idx_or[0, h] = torch.from_numpy(ref_idx).cuda()
+        cnt_or[0, h] = torch.from_numpy(ref_cnt).cuda()
+        sampled[h] = (cubes, toks, rsel, ref_idx, ref_cnt)
+    # fixed-selection path on the oracle's lists
+    out2, oc, of = plan.run_fixed_idx(*dev_in, idx_or, cnt_or, want_coarse=True, want_fine=True)
+    plan.check()
+    for h, (cubes, toks, rsel, ref_idx, ref_cnt) in sampled.items():
+        assert_close(oc[0, h].cpu().numpy(), rsel["Oc"], f"{name} head {h} coarse output", max_abs=1e-4,
+                     mean_abs=1e-5)
+        r = oracle_head(wl, q, k, v, gc, gf, 0, h, query_cubes=cubes, lists_in=ref_idx, counts_in=ref_cnt)
+        t = torch.from_numpy(toks).cuda()
+        assert_close(of[0, h, t].cpu().numpy(), r["Of"][toks], f"{name} head {h} fine output (oracle lists)")
+        assert_close(out2[0, h, t].float().cpu().numpy(), r["out"][toks], f"{name} head {h} gated output (oracle lists)")
     print(f"{name}: exact rows {exact}, exempt rows {exempt} ({exempt / (exact + exempt):.4f})")
     assert exact > 0
 

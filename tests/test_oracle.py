@@ -356,13 +356,14 @@ def test_workloads_match_page_facts():
 def test_forward_tiny_properties():
     wl = synth.WORKLOADS["tiny"]
     q, k, v, gc, gf = synth.make_inputs(wl)
-    out, lists, counts, Oc, Of, S = oracle.forward(q.double().numpy(), k.double().numpy(), v.double().numpy(),
-                                                   gc.double().numpy(), gf.double().numpy(), wl.T, wl.H, wl.W,
-                                                   topk=wl.topk)
-    assert out.shape == (1, 2, 512, 64) and lists.shape == (1, 2, 8, 2)
-    assert np.isfinite(out).all()
-    assert (np.diff(lists, axis=-1) > 0).all()            # ascending, distinct
-    assert (counts == 2).all()
+    for h in range(wl.heads):
+        r = oracle.forward_head(q[0, h].double().numpy(), k[0, h].double().numpy(), v[0, h].double().numpy(),
+                                gc[0, h].double().numpy(), gf[0, h].double().numpy(), wl.T, wl.H, wl.W,
+                                topk=wl.topk)
+        assert r["out"].shape == (512, 64) and r["lists"].shape == (8, 2)
+        assert np.isfinite(r["out"]).all()
+        assert (np.diff(r["lists"], axis=-1) > 0).all()            # ascending, distinct
+        assert (r["counts"] == 2).all()
 
 
 def test_topp_mass_property():
