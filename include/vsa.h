@@ -37,7 +37,11 @@
  *   work is enqueued. A failed kernel launch returns VSA_ERR_CUDA. Errors
  *   detected on the device (a bounded wait that gave up) are recorded in the
  *   plan's workspace and returned by the next vsa_check.
- *   A plan must not be used by two streams at the same time.
+ *   Threads may share a plan: its calls take a per-plan lock for their
+ *   host-side work (tensor-map encoding, launches). The plan has one
+ *   workspace, though, so the device work of two calls on different streams
+ *   without ordering between them races on it: order such calls (one
+ *   stream, or events).
  */
 #ifndef VSA_H_
 #define VSA_H_
@@ -153,7 +157,13 @@ vsa_status vsa_run_host(vsa_plan_t plan, const void* q, const void* k, const voi
  * device memory with cudaMalloc; later calls allocate nothing). At most 16
  * configurations are kept, for the life of the process; a call with a 17th
  * returns VSA_ERR_UNSUPPORTED (use vsa_plan for more). topk > 0 selects top-K;
- * topk == 0 selects top-p with kmin = 4 and kmax = min(128, C). */
+ * topk == 0 selects top-p with kmin = 4 and kmax = min(128, C).
+ * Calls with the same configuration on the same device share one cached
+ * plan and workspace: calls whose device work overlaps (different streams
+ * without ordering, or host threads that do not order their streams) race on
+ * that workspace, so serialise them. Device-side errors (a bounded wait that
+ * gave up) are not reported by this form, which has no plan to pass to
+ * vsa_check; use vsa_plan / vsa_run where they must be seen. */
 vsa_status vsa_forward(const void* q, const void* k, const void* v, const float* gate_c, const float* gate_f,
                        int B, int heads, int T, int H, int W, int D, int topk, float top_p, void* out, int32_t* idx,
                        void* stream);
@@ -167,9 +177,11 @@ vsa_status vsa_forward(const void* q, const void* k, const void* v, const float*
  * VSA_NOALLOC_SCRATCH_BYTES inside libvsa.so, which every GPU that loads
  * the library holds until the process exits.
  * The pages describing the method have no counterpart of this entry point.
- *   - Configurations whose workspace (vsa_workspace_bytes) exceeds
- *     VSA_NOALLOC_SCRATCH_BYTES are rejected with VSA_ERR_UNSUPPORTED before
- *     anything is enqueued.
+ *   - Configurations whose workspace exceeds VSA_NOALLOC_SCRATCH_BYTES are
+ *     rejected with VSA_ERR_UNSUPPORTED before anything is enqueued. The
+ *     workspace here is vsa_workspace_bytes(cfg) less the q_cube region,
+ *     which this entry point never writes: e.g. up to 6 heads of D = 128 at
+ *     16,384 tokens (58.1 MiB) fit, 7 do not.
  *   - The first call on each device looks up the device address of the
  *     array (cudaGetSymbolAddress); make that first call before any stream
  *     capture starts.

@@ -28,6 +28,12 @@ struct HostPath {
 };
 
 struct vsa_plan_s {
+  // Serialises the host-side work of calls on this plan (tensor-map encoding,
+  // launches, the recorded stream), so that two threads sharing a plan never
+  // launch with a map encoded for the other thread's q or out. The workspace
+  // itself is still one per plan: work of calls on different streams without
+  // ordering between them races on it on the device.
+  std::mutex mu;
   vsa_config cfg;
   int BH, N, C, kcap;
   char* ws;
@@ -96,7 +102,10 @@ vsa_status validate(const vsa_config* c) {
   return VSA_OK;
 }
 
-void make_layout(const vsa_config* c, vsa_workspace_layout_t* L) {
+// with_q_cube: reserve the region of q's cube-major copy (only written when a
+// plan asks for it with vsa_set_cube_major_copies; the allocation-free entry
+// point never does, so its layout gives the region zero bytes).
+void make_layout(const vsa_config* c, vsa_workspace_layout_t* L, bool with_q_cube = true) {
   const size_t BH = (size_t)c->B * c->heads, N = (size_t)c->T * c->H * c->W, C = N / 64, D = c->D;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -104,7 +113,7 @@ void make_layout(const vsa_config* c, vsa_workspace_layout_t* L) {
     off = align_up(off + bytes, 1024);
     return o;
   };
-  L->q_cube = take(BH * N * D * 2);
+  L->q_cube = take(with_q_cube ? BH * N * D * 2 : 0);
   L->k_cube = take(BH * N * D * 2);
   L->v_cube = take(BH * N * D * 2);
   L->q_pool = take(BH * C * D * 4);
@@ -191,6 +200,7 @@ vsa_status run_common(vsa_plan_t P, const void* q, const void* k, const void* v,
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return VSA_ERR_ALIGN;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lock(P->mu);
   P->last_stream = st;
   const vsa_config& c = P->cfg;
   char* ws = P->ws;
@@ -373,6 +383,7 @@ vsa_status vsa_run_fixed_idx(vsa_plan_t plan, const void* q, const void* k, cons
 vsa_status vsa_run_host(vsa_plan_t plan, const void* q, const void* k, const void* v, const float* gate_c,
                         const float* gate_f, void* out, int32_t* idx, int32_t* cnt, void* stream) {
   if (!plan || !q || !k || !v || !gate_c || !gate_f || !out || !idx) return VSA_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(plan->mu);
   const int n = plan->BH;
   HostPath* H = plan->host;
   if (!H) {
@@ -541,7 +552,7 @@ vsa_status vsa_forward_noalloc(const void* q, const void* k, const void* v, cons
   if (s != VSA_OK) return s;
   if (!out || !idx) return VSA_ERR_INVALID_ARG;
   vsa_workspace_layout_t L;
-  make_layout(&cfg, &L);
+  make_layout(&cfg, &L, /*with_q_cube=*/false);
   if (L.total > VSA_NOALLOC_SCRATCH_BYTES) return VSA_ERR_UNSUPPORTED;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return VSA_ERR_CUDA;
@@ -580,7 +591,12 @@ vsa_status vsa_check(vsa_plan_t plan) {
     const vsa_status hs = vsa_check(plan->host->sub);
     if (hs != VSA_OK) return hs;
   }
-  if (cudaStreamSynchronize(plan->last_stream) != cudaSuccess) return VSA_ERR_CUDA;
+  cudaStream_t last;
+  {
+    std::lock_guard<std::mutex> lock(plan->mu);
+    last = plan->last_stream;
+  }
+  if (cudaStreamSynchronize(last) != cudaSuccess) return VSA_ERR_CUDA;
   int err = 0;
   int* dev_err = reinterpret_cast<int*>(plan->ws + plan->lay.err);
   if (cudaMemcpy(&err, dev_err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return VSA_ERR_CUDA;

@@ -15,12 +15,18 @@
 // hi.hi, hi.mid, mid.hi, mid.mid, hi.lo, lo.hi in fp32 tensor memory; the
 // dropped ones are below 2^-24 relative.
 //   1. scores   s = qbar kbar^T / sqrt(D)       [BH, C, C]   (tcgen05, 128 x 128 tiles)
-//   2. select   row max / sum, exact K-th largest score by a 32-step radix
-//               search on order-preserving integer keys (one warp per row,
-//               keys in registers), ascending index lists with ties to the
-//               lower id; top-p ranks the kmax best candidates and cuts at
-//               the first prefix whose mass reaches p. Writes P as three
-//               bf16 terms.
+//   2. select   one warp per row, the row's scores as order-preserving
+//               uint32 keys in shared memory: row max and sum, the
+//               probabilities P written as three bf16 terms, then the
+//               selection. Top-K <= 32: the minimum of the lanes' maxima
+//               bounds the K-th largest key from below, the keys at or above
+//               it are compacted in place (ascending id) and an MSB-first
+//               count search over them finds the K-th largest; larger K, or
+//               more than 256 candidates, search over all keys. Top-p (own
+//               kernel): the exact kmax-th largest key by the same search,
+//               the kmax candidates ranked by (score desc, id asc) and cut at
+//               the first prefix whose mass reaches p, clamped to
+//               [kmin, kmax]. Lists are ascending, ties go to the lower id.
 //   3. output   Oc = P vbar                     [BH, C, D]   (tcgen05, 128 x D tiles)
 #include "sm100_ptx.cuh"
 #include "vsa_common.cuh"

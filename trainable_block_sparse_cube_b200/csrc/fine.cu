@@ -53,6 +53,7 @@
 // records kErrTimeout, sets a CTA-wide abort flag that makes every later wait
 // return at once, and the CTA then drains its own in-flight TMA copies and
 // MMAs before releasing TMEM and exiting.
+#include "poly_exp2.cuh"
 #include "sm100_ptx.cuh"
 #include "vsa_common.cuh"
 
@@ -131,22 +132,6 @@ __device__ __forceinline__ void st_16x128b_x8(uint32_t taddr, const uint32_t (&r
 }
 #undef VSA_O4
 #undef VSA_I4
-
-// 2^x on the FMA pipe, for x in [-126, 64] (clamped): x = n + f with n the
-// nearest integer (added to 1.5 * 2^23 so that it lands in the low mantissa
-// bits) and f in [-1/2, 1/2]; 2^f is a cubic fitted by weighted least squares
-// (relative error) on Chebyshev nodes of [-1/2, 1/2], max relative error
-// 7.8e-5, far below the bf16 rounding of P; 2^n is added to the exponent
-// field. Offloads part of the exponentials from the MUFU units.
-__device__ __forceinline__ float poly_exp2(float x) {
-  x = fminf(fmaxf(x, -126.f), 64.f);
-  const float t = __fadd_rn(x, 12582912.f);
-  const float f = __fsub_rn(x, __fsub_rn(t, 12582912.f));
-  float p = fmaf(0.05508868396282196f, f, 0.24260404706001282f);
-  p = fmaf(p, f, 0.6932762265205383f);
-  p = fmaf(p, f, 0.9999289512634277f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
 
 // Softmax numerators of one 64-key half step for the thread's rows a and a+8
 // (register layout of ld_16x256b_x8): P = 2^(s*scale - m), packed to bf16
