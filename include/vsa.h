@@ -247,6 +247,17 @@ vsa_status vsa_stage_times(vsa_plan_t plan, float* ms);
 /* Number of kernel launches one vsa_run / vsa_run_fixed_idx call makes. */
 int vsa_kernels_per_run(void);
 
+/* Measurement hook (not a step of the method; the pages have no counterpart):
+ * enqueues one kernel that reads the first floor(bytes / 16384) * 16384
+ * bytes of the device buffer `buf` `passes` times, in 16 KB untiled bulk
+ * copies into shared memory (the TMA engine, as the fine-attention kernel
+ * loads its K/V tiles), two CTAs per SM. Time it with events on `stream`;
+ * with a buffer that fits in L2 (and a first pass to bring it there) the
+ * rate is the L2 -> SM bandwidth of such copies. Nothing is written except
+ * *status (a device int the caller zeroes): bit 0 is set if a bounded wait
+ * gave up. buf and status must be 16-byte aligned; bytes >= 16384. */
+vsa_status vsa_measure_l2_read(const void* buf, size_t bytes, int passes, int* status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

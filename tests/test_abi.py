@@ -24,7 +24,7 @@ def _declared_functions():
     for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
         text = open(h).read()
         text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-        names += re.findall(r"\b(vsa_[a-z_]+)\s*\(", text)
+        names += re.findall(r"\b(vsa_[a-z0-9_]+)\s*\(", text)
     return sorted(set(names))
 
 

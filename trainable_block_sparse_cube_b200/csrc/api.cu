@@ -657,6 +657,18 @@ vsa_status vsa_stage_times(vsa_plan_t plan, float* ms) {
 
 int vsa_kernels_per_run(void) { return 5; }
 
+vsa_status vsa_measure_l2_read(const void* buf, size_t bytes, int passes, int* status, void* stream) {
+  if (!buf || !status || passes < 1 || bytes < 16384) return VSA_ERR_INVALID_ARG;
+  if (!aligned16(buf) || !aligned16(status)) return VSA_ERR_ALIGN;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return VSA_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return VSA_ERR_CUDA;
+  return vsa::launch_l2_read(buf, bytes, passes, status, 2 * sms, reinterpret_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? VSA_OK
+             : VSA_ERR_CUDA;
+}
+
 vsa_status vsa_set_debug_stall(vsa_plan_t plan, int on) {
   if (!plan) return VSA_ERR_INVALID_ARG;
   plan->debug_stall = on ? 1 : 0;

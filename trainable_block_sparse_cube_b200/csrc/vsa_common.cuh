@@ -75,5 +75,6 @@ struct FineParams {
 cudaError_t launch_gather(const GatherParams& p, int D, cudaStream_t st);
 cudaError_t launch_coarse(const CoarseParams& p, cudaStream_t st);
 cudaError_t launch_fine(const FineParams& p, int D, int grid, cudaStream_t st);
+cudaError_t launch_l2_read(const void* buf, size_t bytes, int passes, int* status, int grid, cudaStream_t st);
 
 }  // namespace vsa

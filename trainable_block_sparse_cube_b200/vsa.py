@@ -21,7 +21,7 @@ STATUS = {0: "VSA_OK", 1: "VSA_ERR_INVALID_ARG", 2: "VSA_ERR_SHAPE", 3: "VSA_ERR
 EXPORTED = ["vsa_workspace_bytes", "vsa_workspace_layout", "vsa_plan", "vsa_run", "vsa_run_fixed_idx",
             "vsa_forward", "vsa_check", "vsa_plan_destroy", "vsa_status_string", "vsa_set_wait_limit_ns",
             "vsa_set_debug_stall", "vsa_set_stage_timing", "vsa_stage_times", "vsa_kernels_per_run",
-            "vsa_forward_noalloc", "vsa_set_cube_major_copies", "vsa_run_host"]
+            "vsa_forward_noalloc", "vsa_set_cube_major_copies", "vsa_run_host", "vsa_measure_l2_read"]
 
 
 class VSAError(RuntimeError):
@@ -88,6 +88,8 @@ def load():
     L.vsa_kernels_per_run.restype = i32
     L.vsa_forward_noalloc.argtypes = [vp] * 5 + [i32] * 7 + [ctypes.c_float, vp, vp, vp]
     L.vsa_forward_noalloc.restype = i32
+    L.vsa_measure_l2_read.argtypes = [vp, sz, i32, vp, vp]
+    L.vsa_measure_l2_read.restype = i32
     _lib = L
     return L
 
@@ -246,6 +248,16 @@ class Plan:
 
     def pooled(self, which: str):
         return self.workspace_view(f"{which}_pool", torch.float32, (self.B * self.heads, self.C, self.D))
+
+
+def measure_l2_read(buf, passes, status):
+    """Enqueues the L2 -> SM bulk-copy read of the uint8 CUDA tensor `buf`
+    (`passes` times) on the current stream; `status` is a zeroed int32 CUDA
+    tensor (bit 0 set if a bounded wait gave up)."""
+    _need(buf, "buf", torch.uint8, tuple(buf.shape))
+    _need(status, "status", torch.int32, tuple(status.shape))
+    _check(load().vsa_measure_l2_read(_ptr(buf), buf.numel(), int(passes), _ptr(status), _stream()),
+           "vsa_measure_l2_read")
 
 
 def forward(q, k, v, gate_c, gate_f, T, H, W, topk=0, top_p=0.0, out=None, idx=None):
