@@ -129,6 +129,58 @@ vsa_status vsa_run_fixed_idx(vsa_plan_t plan, const void* q, const void* k, cons
                              const float* gate_f, const int32_t* idx_in, const int32_t* cnt_in, void* out,
                              float* out_coarse, float* out_fine, void* stream);
 
+/* Training forward pass: vsa_run, and it also saves what vsa_run_backward
+ * needs ("Faster Video Diffusion with Trainable Sparse Attention",
+ * "Approach": the hierarchy is trained end to end; "VSA: Faster Video
+ * Diffusion with Trainable Sparse Attention", "Abstract (arXiv)": a single
+ * differentiable kernel).
+ *   o_fine: [B,heads,N,D] bf16, written: the fine-attention output before
+ *           gating (raster order).
+ *   lse:    [B,heads,N] fp32, written: per token n, the natural log of its
+ *           fine softmax denominator, log(sum_m exp(q_n . k_m / sqrt(D))) over
+ *           the tokens m of its query cube's selected cubes (raster order).
+ *   out, idx, cnt as in vsa_run (cnt may be NULL). */
+vsa_status vsa_run_train(vsa_plan_t plan, const void* q, const void* k, const void* v, const float* gate_c,
+                         const float* gate_f, void* out, int32_t* idx, int32_t* cnt, void* o_fine, float* lse,
+                         void* stream);
+
+/* Bytes of device workspace vsa_run_backward needs for cfg (0 if cfg is
+ * invalid): dO in cube-major order, per-token statistics, the coarse
+ * backward's C x C products and the transposed selection lists. */
+size_t vsa_backward_workspace_bytes(const vsa_config* cfg);
+
+/* Backward pass of the forward pass with the selection held fixed (an index
+ * choice has no gradient; the pages give no gradient formulas, so these are
+ * the chain rule of the forward computation):
+ *   dgate_c[n] = dout_n . Oc[cube(n)]          dgate_f[n] = dout_n . Of_n
+ *   fine (per query cube i over the tokens of its selected cubes, with
+ *   dOf = gate_f dout, P = exp(q k^T/sqrt(D) - lse), delta_n = dOf_n . Of_n):
+ *     dS = P o (dOf v^T - delta); dq = dS k / sqrt(D); dk = dS^T q / sqrt(D);
+ *     dv = P^T dOf, the key and value terms summed over every query cube
+ *     that selected the cube;
+ *   coarse (dense over the pooled tokens, dOc[c] = sum over cube c's tokens
+ *   of gate_c dout): the attention gradient of the means, handed to every
+ *   token of a cube with weight 1/64 (the mean's derivative).
+ * Inputs: q, k, v, gate_c, gate_f as given to vsa_run_train; idx, cnt the
+ *   selection it returned (cnt may be NULL in top-K mode; every row must be
+ *   strictly ascending, ids in [0, C), counts in [1, Kcap]); o_fine and lse
+ *   the tensors it saved; dout [B,heads,N,D] bf16, the gradient of out.
+ * Outputs (written): dq, dk, dv [B,heads,N,D] bf16; dgate_c, dgate_f
+ *   [B,heads,N] fp32.
+ * bwd_workspace: device memory of at least vsa_backward_workspace_bytes(cfg)
+ *   bytes, 256-byte aligned, owned by the caller. The call also recomputes
+ *   the gather and the coarse stage into the plan's workspace (so the plan's
+ *   workspace contents of an earlier forward call are overwritten).
+ * Two kernels compute the fine gradients without atomics (query-major dq,
+ * KV-major dk and dv), so the results are deterministic. A malformed
+ * selection (id out of range, a row not strictly ascending, a count outside
+ * [1, Kcap]) is never used as an address; it is reported by vsa_check as
+ * VSA_ERR_INVALID_ARG and its gradients are then unspecified. */
+vsa_status vsa_run_backward(vsa_plan_t plan, void* bwd_workspace, size_t bwd_bytes, const void* q, const void* k,
+                            const void* v, const float* gate_c, const float* gate_f, const int32_t* idx,
+                            const int32_t* cnt, const void* o_fine, const float* lse, const void* dout, void* dq,
+                            void* dk, void* dv, float* dgate_c, float* dgate_f, void* stream);
+
 /* Forward pass on HOST buffers: copies the inputs to the device, runs the
  * forward pass (as vsa_run) and copies the results back, all enqueued on
  * `stream`. The pages describing the method have no counterpart of this
@@ -233,16 +285,29 @@ vsa_status vsa_set_debug_stall(vsa_plan_t plan, int on);
  * write q's copy into region q_cube (one extra write of q); off by default. */
 vsa_status vsa_set_cube_major_copies(vsa_plan_t plan, int on);
 
-/* Stage timing for benchmarks. When `on` is nonzero, later runs of this plan
- * record CUDA events (created here, once) on the run's stream around its three
- * stages: gather + pool, coarse attention + selection, fine attention +
- * combine. */
+/* Stage timing for benchmarks. When `on` is positive, later runs of this plan
+ * record CUDA events on the run's stream around its three stages: gather +
+ * pool, coarse attention + selection, fine attention + combine; the events of
+ * the last `on` runs are kept (at most 4096; created here). 0 switches timing
+ * off. Every call restarts the count of recorded runs. */
 vsa_status vsa_set_stage_timing(vsa_plan_t plan, int on);
 
 /* Waits for the events of the last timed run and writes the device time of
  * its stages in milliseconds to ms[0] (gather + pool), ms[1] (coarse),
  * ms[2] (fine). VSA_ERR_INVALID_ARG if timing is off or nothing ran yet. */
 vsa_status vsa_stage_times(vsa_plan_t plan, float* ms);
+
+/* The stage times of the last min(max_runs, runs kept) timed runs, oldest
+ * first: ms[3 i + s] for run i and stage s (as in vsa_stage_times); the
+ * number of runs written goes to *n_runs. Waits for the last run's events. */
+vsa_status vsa_stage_times_history(vsa_plan_t plan, float* ms, int max_runs, int* n_runs);
+
+/* Waits for the events of the last timed vsa_run_backward and writes the
+ * device time of its stages in milliseconds: ms[0] gather + coarse forward
+ * (recomputed), ms[1] per-token preparation + transposed lists + coarse
+ * backward, ms[2] fine dq, ms[3] fine dk / dv. VSA_ERR_INVALID_ARG if timing
+ * is off or no backward ran since it was switched on. */
+vsa_status vsa_backward_stage_times(vsa_plan_t plan, float* ms);
 
 /* Number of kernel launches one vsa_run / vsa_run_fixed_idx call makes. */
 int vsa_kernels_per_run(void);

@@ -25,7 +25,7 @@ import numpy as np
 
 from .vsa_oracle import coarse_attention, cube_perm, fine_attention, pool_cubes
 
-__all__ = ["attention_backward", "backward_head"]
+__all__ = ["attention_backward", "backward_head", "fine_lse"]
 
 
 def attention_backward(q: np.ndarray, k: np.ndarray, v: np.ndarray, dout: np.ndarray, scale: float):
@@ -45,7 +45,29 @@ def attention_backward(q: np.ndarray, k: np.ndarray, v: np.ndarray, dout: np.nda
     return dS @ k * scale, dS.T @ q * scale, dv
 
 
-def backward_head(q, k, v, gate_c, gate_f, dout, T, H, W, lists, counts):
+def fine_lse(q: np.ndarray, k: np.ndarray, perm: np.ndarray, lists: np.ndarray, counts: np.ndarray,
+             query_cubes=None) -> np.ndarray:
+    """Per query token n, the natural log of its fine softmax denominator,
+    log sum_m exp(q_n . k_m / sqrt(D)) over the tokens m of its query cube's
+    selected cubes (the normaliser of the fine attention in vsa_oracle.py, the
+    forward statistic the backward pass reuses). Raster order [N]; tokens of
+    query cubes not in `query_cubes` are NaN.
+    Pinned by: torch.logsumexp over the masked logits (-inf outside the
+    selection), and exp(logits - lse) rows summing to one.
+    """
+    N, D = q.shape
+    C = N // 64
+    cube_tok = perm.reshape(C, 64)
+    out = np.full(N, np.nan)
+    for i in (range(C) if query_cubes is None else query_cubes):
+        kv_tok = cube_tok[lists[i, : counts[i]]].reshape(-1)
+        logits = (q[cube_tok[i]] @ k[kv_tok].T) / math.sqrt(D)
+        m = logits.max(axis=1)
+        out[cube_tok[i]] = m + np.log(np.exp(logits - m[:, None]).sum(axis=1))
+    return out
+
+
+def backward_head(q, k, v, gate_c, gate_f, dout, T, H, W, lists, counts, query_cubes=None, kv_cubes=None):
     """Gradients of one (batch, head) of the gated forward pass.
 
     Forward (vsa_oracle.forward_head with the selection `lists`/`counts`):
@@ -61,7 +83,13 @@ def backward_head(q, k, v, gate_c, gate_f, dout, T, H, W, lists, counts):
       pooling: every token of cube c receives 1/64 of the mean's gradient.
     Inputs [N, D] and [N] in raster order, fp64. Returns a dict with
     dq, dk, dv [N, D] and dgate_c, dgate_f [N].
-    Pinned by: central finite differences of the forward oracle.
+    query_cubes / kv_cubes (optional) restrict the work to sampled outputs:
+    dq only for the tokens of query_cubes, dk and dv only for the tokens of
+    kv_cubes (each still summed over every query cube that selected it); the
+    other rows of those arrays are NaN. The fine terms are the only ones
+    restricted; the result on the sampled rows is the same.
+    Pinned by: central finite differences of the forward oracle; the sampled
+    rows equal the unrestricted result.
     """
     N, D = q.shape
     C = N // 64
@@ -84,8 +112,15 @@ def backward_head(q, k, v, gate_c, gate_f, dout, T, H, W, lists, counts):
     dq = np.zeros((N, D))
     dk = np.zeros((N, D))
     dv = np.zeros((N, D))
+    qset = None if query_cubes is None else set(int(x) for x in query_cubes)
+    kvset = None if kv_cubes is None else set(int(x) for x in kv_cubes)
     for i in range(C):
-        kv_tok = cube_tok[lists[i, : counts[i]]].reshape(-1)
+        sel = lists[i, : counts[i]]
+        want_q = qset is None or i in qset
+        want_kv = kvset is None or any(int(j) in kvset for j in sel)
+        if not (want_q or want_kv):
+            continue
+        kv_tok = cube_tok[sel].reshape(-1)
         qi = cube_tok[i]
         gq, gk, gv = attention_backward(q[qi], k[kv_tok], v[kv_tok], dOf[qi], scale)
         dq[qi] += gq
@@ -96,4 +131,10 @@ def backward_head(q, k, v, gate_c, gate_f, dout, T, H, W, lists, counts):
     dq += gqb[cube_of] / 64.0
     dk += gkb[cube_of] / 64.0
     dv += gvb[cube_of] / 64.0
+    if qset is not None:
+        dq[~np.isin(cube_of, list(qset))] = np.nan
+    if kvset is not None:
+        keep = np.isin(cube_of, list(kvset))
+        dk[~keep] = np.nan
+        dv[~keep] = np.nan
     return dict(dq=dq, dk=dk, dv=dv, dgate_c=dgate_c, dgate_f=dgate_f)

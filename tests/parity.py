@@ -106,3 +106,25 @@ def assert_close(gpu, ref, what, max_abs=MAX_ABS, mean_abs=MEAN_ABS):
     assert d.max() <= max_abs and d.mean() <= mean_abs, \
         f"{what}: max abs {d.max():.3e} (<= {max_abs}), mean abs {d.mean():.3e} (<= {mean_abs})"
     return float(d.max()), float(d.mean())
+
+
+# Gradients are compared relative to their own scale: with N(0, 1) upstream
+# gradients their magnitudes are ~1e-2, so the forward's absolute bounds would
+# pin nothing. The error is measured in units of the reference's RMS over the
+# compared elements.
+GRAD_MAX_REL = 3e-2
+GRAD_MEAN_REL = 5e-3
+
+
+def assert_close_rel(gpu, ref, what, max_rel=GRAD_MAX_REL, mean_rel=GRAD_MEAN_REL):
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert gpu.shape == ref.shape, (what, gpu.shape, ref.shape)
+    assert np.isfinite(gpu).all(), f"{what}: non-finite values"
+    rms = float(np.sqrt(np.mean(ref * ref)))
+    assert rms > 0, f"{what}: reference is zero"
+    d = np.abs(gpu - ref) / rms
+    print(f"{what}: max {d.max():.2e} mean {d.mean():.2e} (x rms {rms:.2e})")
+    assert d.max() <= max_rel and d.mean() <= mean_rel, \
+        f"{what}: max {d.max():.3e} (<= {max_rel}), mean {d.mean():.3e} (<= {mean_rel}) in units of rms {rms:.3e}"
+    return float(d.max()), float(d.mean())

@@ -13,7 +13,7 @@ import pytest
 import torch
 
 import oracle
-from oracle.vsa_oracle_backward import attention_backward, backward_head
+from oracle.vsa_oracle_backward import attention_backward, backward_head, fine_lse
 
 T = H = W = 8          # 512 tokens, 8 cubes
 D = 8
@@ -86,3 +86,44 @@ def test_zero_fine_gate_leaves_only_the_coarse_path():
         per_cube = g[name][perm].reshape(-1, 64, D)
         assert np.allclose(per_cube, per_cube[:, :1, :], atol=1e-14)
     assert np.allclose(g["dgate_f"], (dout * r["Of"]).sum(axis=1))
+
+
+def test_fine_lse_matches_torch_logsumexp():
+    q, k, v, gc, gf, dout = _inputs(11)
+    r = oracle.forward_head(q, k, v, gc, gf, T, H, W, topk=K)
+    perm = oracle.cube_perm(T, H, W)
+    counts = np.array([1, 2, 3, 1, 3, 2, 1, 3])
+    lse = fine_lse(q, k, perm, r["lists"], counts)
+    N = T * H * W
+    cube_of = np.empty(N, dtype=np.int64)
+    cube_of[perm] = np.arange(N) // 64
+    # torch.logsumexp over the full logits with -inf outside each token's selection
+    mask = np.zeros((N, N), dtype=bool)
+    for n in range(N):
+        for j in r["lists"][cube_of[n], : counts[cube_of[n]]]:
+            mask[n, perm[64 * j: 64 * j + 64]] = True
+    logits = torch.from_numpy(q @ k.T / math.sqrt(D)).masked_fill(torch.from_numpy(~mask), float("-inf"))
+    ref = torch.logsumexp(logits, dim=1).numpy()
+    assert np.allclose(lse, ref, rtol=1e-12, atol=1e-12)
+    # the softmax rebuilt from lse sums to one over the selection
+    assert np.allclose(np.where(mask, np.exp(logits.numpy() - lse[:, None]), 0).sum(axis=1), 1.0)
+    # a planted mistake (missing 1/sqrt(D)) fails the pin
+    bad = fine_lse(q * math.sqrt(D), k, perm, r["lists"], counts)
+    assert not np.allclose(bad, ref, rtol=1e-6)
+
+
+def test_sampled_backward_equals_full_on_sampled_rows():
+    q, k, v, gc, gf, dout = _inputs(5)
+    r = oracle.forward_head(q, k, v, gc, gf, T, H, W, topk=K)
+    counts = np.array([1, 2, 3, 1, 3, 2, 1, 3])
+    full = backward_head(q, k, v, gc, gf, dout, T, H, W, r["lists"], counts)
+    part = backward_head(q, k, v, gc, gf, dout, T, H, W, r["lists"], counts, query_cubes=[1, 6], kv_cubes=[0, 5])
+    perm = oracle.cube_perm(T, H, W)
+    cube_of = np.empty(T * H * W, dtype=np.int64)
+    cube_of[perm] = np.arange(T * H * W) // 64
+    qrows = np.isin(cube_of, [1, 6])
+    kvrows = np.isin(cube_of, [0, 5])
+    assert np.array_equal(part["dq"][qrows], full["dq"][qrows]) or np.allclose(part["dq"][qrows], full["dq"][qrows])
+    assert np.allclose(part["dk"][kvrows], full["dk"][kvrows], rtol=1e-13, atol=1e-13)
+    assert np.allclose(part["dv"][kvrows], full["dv"][kvrows], rtol=1e-13, atol=1e-13)
+    assert np.isnan(part["dq"][~qrows]).all() and np.isnan(part["dk"][~kvrows]).all()

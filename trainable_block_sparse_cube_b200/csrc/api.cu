@@ -41,6 +41,7 @@ struct vsa_plan_s {
   CUtensorMap tm_q;         // raster map of q, encoded for the pointer tm_q_for
   const void* tm_q_for;
   CUtensorMap tm_k, tm_v;   // maps over the cube-major copies in the workspace
+  CUtensorMap tm_qc;        // map over q's cube-major copy (written by the backward pass's gather)
   CUtensorMap tm_qs, tm_ks, tm_vs, tm_ps;  // maps over the coarse operands' bf16 terms
   CUtensorMap tm_out;       // output map, encoded for the output pointer tm_out_for
   const void* tm_out_for;
@@ -51,7 +52,10 @@ struct vsa_plan_s {
   int debug_stall;
   int timing;        // record stage events
   int timed_runs;    // runs recorded since timing was enabled
-  cudaEvent_t ev[4];
+  cudaEvent_t* ev;     // stage events of the forward: 4 per run, for the last `ring` runs
+  int ring;            // runs kept (vsa_set_stage_timing)
+  cudaEvent_t evb[5];  // backward stages: prologue, prep + lists + coarse, dQ, dK/dV
+  int timed_bwd;       // backward runs recorded since timing was enabled
   HostPath* host;    // vsa_run_host state (null until its first call)
 };
 
@@ -90,6 +94,7 @@ vsa_status validate(const vsa_config* c) {
   const long long C = N / 64;
   if (C > kMaxC) return VSA_ERR_UNSUPPORTED;
   if ((long long)c->B * c->heads * N * c->D >= (1LL << 40)) return VSA_ERR_UNSUPPORTED;
+  if ((long long)c->B * c->heads * N >= (1LL << 31)) return VSA_ERR_UNSUPPORTED;  // TMA row coordinates
   if ((long long)c->B * c->heads > 65535) return VSA_ERR_UNSUPPORTED;
   if (c->topk < 0) return VSA_ERR_INVALID_ARG;
   if (c->topk > 0) {
@@ -125,6 +130,35 @@ void make_layout(const vsa_config* c, vsa_workspace_layout_t* L, bool with_q_cub
   L->p_split = take(3 * BH * C * coarse_pitch(C) * 2);
   L->cnt = take(BH * C * 4);
   L->err = take(16);
+  L->total = off;
+}
+
+// Regions of the backward pass's workspace (byte offsets).
+struct BwdLayout {
+  size_t do_cube, qstat, doc, dlc, p32, ds, dqbar, dkbar, dvbar, bitmap, tcnt, toff, tlist, total;
+};
+void make_bwd_layout(const vsa_config* c, BwdLayout* L) {
+  const size_t BH = (size_t)c->B * c->heads, N = (size_t)c->T * c->H * c->W, C = N / 64, D = c->D;
+  const size_t kcap = c->topk > 0 ? (size_t)c->topk : (size_t)c->kmax, W32 = (C + 31) / 32;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 1024);
+    return o;
+  };
+  L->do_cube = take(BH * N * D * 2);
+  L->qstat = take(BH * C * 128 * 4);
+  L->doc = take(BH * C * D * 4);
+  L->dlc = take(BH * C * 4);
+  L->p32 = take(BH * C * C * 4);
+  L->ds = take(BH * C * C * 4);
+  L->dqbar = take(BH * C * D * 4);
+  L->dkbar = take(BH * C * D * 4);
+  L->dvbar = take(BH * C * D * 4);
+  L->bitmap = take(BH * C * W32 * 4);
+  L->tcnt = take(BH * C * 4);
+  L->toff = take(BH * C * 4);
+  L->tlist = take(BH * C * kcap * 4);
   L->total = off;
 }
 
@@ -192,11 +226,13 @@ vsa_status encode_raster_map(CUtensorMap* m, const void* base, const vsa_config&
 
 vsa_status run_common(vsa_plan_t P, const void* q, const void* k, const void* v, const float* gate_c,
                       const float* gate_f, bool select, const int32_t* idx_in, const int32_t* cnt_in, int32_t* idx_out,
-                      int32_t* cnt_out, void* out, float* out_coarse, float* out_fine, void* stream) {
+                      int32_t* cnt_out, void* out, float* out_coarse, float* out_fine, void* stream,
+                      void* o_fine = nullptr, float* lse = nullptr) {
   if (!P || !q || !k || !v || !gate_c || !gate_f) return VSA_ERR_INVALID_ARG;
   if (select && !idx_out) return VSA_ERR_INVALID_ARG;
   if (!select && !idx_in) return VSA_ERR_INVALID_ARG;
-  const void* ptrs[] = {q, k, v, gate_c, gate_f, idx_in, cnt_in, idx_out, cnt_out, out, out_coarse, out_fine};
+  const void* ptrs[] = {q, k, v, gate_c, gate_f, idx_in, cnt_in, idx_out, cnt_out, out, out_coarse, out_fine,
+                        o_fine, lse};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return VSA_ERR_ALIGN;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -219,9 +255,10 @@ vsa_status run_common(vsa_plan_t P, const void* q, const void* k, const void* v,
   for (int t = 0; t < 3; ++t)
     gp.split[t] = reinterpret_cast<__nv_bfloat16*>(ws + L.pool_split + (size_t)t * 3 * P->BH * P->C * c.D * 2);
   gp.BH = P->BH; gp.C = P->C; gp.H = c.H; gp.W = c.W; gp.N = P->N;
-  if (P->timing && cudaEventRecord(P->ev[0], st) != cudaSuccess) return VSA_ERR_CUDA;
+  cudaEvent_t* ev = P->timing ? P->ev + 4 * (P->timed_runs % P->ring) : nullptr;
+  if (ev && cudaEventRecord(ev[0], st) != cudaSuccess) return VSA_ERR_CUDA;
   if (vsa::launch_gather(gp, c.D, st) != cudaSuccess) return VSA_ERR_CUDA;
-  if (P->timing && cudaEventRecord(P->ev[1], st) != cudaSuccess) return VSA_ERR_CUDA;
+  if (ev && cudaEventRecord(ev[1], st) != cudaSuccess) return VSA_ERR_CUDA;
 
   vsa::CoarseParams cp{};
   cp.tm_qs = P->tm_qs; cp.tm_ks = P->tm_ks; cp.tm_vs = P->tm_vs; cp.tm_ps = P->tm_ps;
@@ -262,6 +299,8 @@ vsa_status run_common(vsa_plan_t P, const void* q, const void* k, const void* v,
   fp.gate_c = gate_c; fp.gate_f = gate_f;
   fp.out = static_cast<__nv_bfloat16*>(out);
   fp.out_fine = out_fine;
+  fp.o_fine = static_cast<__nv_bfloat16*>(o_fine);
+  fp.lse = lse;
   fp.err = reinterpret_cast<int*>(ws + L.err);
   fp.wait_ns = P->wait_ns;
   fp.BH = P->BH; fp.C = P->C; fp.H = c.H; fp.W = c.W; fp.N = P->N;
@@ -269,10 +308,10 @@ vsa_status run_common(vsa_plan_t P, const void* q, const void* k, const void* v,
   fp.scale_log2 = 1.4426950408889634f / std::sqrt((float)c.D);
   fp.debug_stall = P->debug_stall;
   const int grid = fp.n_items < P->num_sms ? fp.n_items : P->num_sms;
-  if (P->timing && cudaEventRecord(P->ev[2], st) != cudaSuccess) return VSA_ERR_CUDA;
+  if (ev && cudaEventRecord(ev[2], st) != cudaSuccess) return VSA_ERR_CUDA;
   if (vsa::launch_fine(fp, c.D, grid, st) != cudaSuccess) return VSA_ERR_CUDA;
   if (P->timing) {
-    if (cudaEventRecord(P->ev[3], st) != cudaSuccess) return VSA_ERR_CUDA;
+    if (cudaEventRecord(ev[3], st) != cudaSuccess) return VSA_ERR_CUDA;
     P->timed_runs++;
   }
 
@@ -280,6 +319,134 @@ vsa_status run_common(vsa_plan_t P, const void* q, const void* k, const void* v,
     if (cudaMemcpyAsync(cnt_out, cp.cnt, (size_t)P->BH * P->C * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
       return VSA_ERR_CUDA;
   }
+  return VSA_OK;
+}
+
+// Backward pass (see include/vsa.h, vsa_run_backward): the gather (with q's
+// cube-major copy) and the coarse stage are recomputed into the plan's
+// workspace, then prep, transposed lists, the coarse backward, and the two
+// fine backward kernels run with the backward workspace.
+vsa_status run_backward(vsa_plan_t P, void* bws, size_t bws_bytes, const void* q, const void* k, const void* v,
+                        const float* gate_c, const float* gate_f, const int32_t* idx, const int32_t* cnt,
+                        const void* o_fine, const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                        float* dgate_c, float* dgate_f, void* stream) {
+  if (!P || !bws || !q || !k || !v || !gate_c || !gate_f || !idx || !o_fine || !lse || !dout || !dq || !dk || !dv ||
+      !dgate_c || !dgate_f)
+    return VSA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, gate_c, gate_f, idx, cnt, o_fine, lse, dout, dq, dk, dv, dgate_c, dgate_f};
+  for (const void* x : ptrs)
+    if (x && !aligned16(x)) return VSA_ERR_ALIGN;
+  if (reinterpret_cast<uintptr_t>(bws) & 255u) return VSA_ERR_ALIGN;
+  BwdLayout BL;
+  make_bwd_layout(&P->cfg, &BL);
+  if (bws_bytes < BL.total) return VSA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lock(P->mu);
+  P->last_stream = st;
+  const vsa_config& c = P->cfg;
+  const int D = c.D;
+  char* ws = P->ws;
+  char* bw = static_cast<char*>(bws);
+  const vsa_workspace_layout_t& L = P->lay;
+  const bool timing = P->timing && P->evb[0];
+  auto mark = [&](int i) { return !timing || cudaEventRecord(P->evb[i], st) == cudaSuccess; };
+
+  // 1. gather + pool (with q's cube-major copy), coarse attention without selection
+  if (!mark(0)) return VSA_ERR_CUDA;
+  vsa::GatherParams gp{};
+  gp.src[0] = static_cast<const __nv_bfloat16*>(q);
+  gp.src[1] = static_cast<const __nv_bfloat16*>(k);
+  gp.src[2] = static_cast<const __nv_bfloat16*>(v);
+  gp.dst[0] = reinterpret_cast<__nv_bfloat16*>(ws + L.q_cube);
+  gp.dst[1] = reinterpret_cast<__nv_bfloat16*>(ws + L.k_cube);
+  gp.dst[2] = reinterpret_cast<__nv_bfloat16*>(ws + L.v_cube);
+  gp.pool[0] = reinterpret_cast<float*>(ws + L.q_pool);
+  gp.pool[1] = reinterpret_cast<float*>(ws + L.k_pool);
+  gp.pool[2] = reinterpret_cast<float*>(ws + L.v_pool);
+  for (int t = 0; t < 3; ++t)
+    gp.split[t] = reinterpret_cast<__nv_bfloat16*>(ws + L.pool_split + (size_t)t * 3 * P->BH * P->C * D * 2);
+  gp.BH = P->BH; gp.C = P->C; gp.H = c.H; gp.W = c.W; gp.N = P->N;
+  if (vsa::launch_gather(gp, D, st) != cudaSuccess) return VSA_ERR_CUDA;
+  vsa::CoarseParams cp{};
+  cp.tm_qs = P->tm_qs; cp.tm_ks = P->tm_ks; cp.tm_vs = P->tm_vs; cp.tm_ps = P->tm_ps;
+  cp.psplit = reinterpret_cast<__nv_bfloat16*>(ws + L.p_split);
+  cp.Cp = (int)coarse_pitch(P->C);
+  cp.err = reinterpret_cast<int*>(ws + L.err);
+  cp.wait_ns = P->wait_ns;
+  cp.s = reinterpret_cast<float*>(ws + L.s_coarse);
+  cp.oc = reinterpret_cast<float*>(ws + L.o_coarse);
+  cp.cnt = reinterpret_cast<int32_t*>(ws + L.cnt);
+  cp.BH = P->BH; cp.C = P->C; cp.D = D; cp.kcap = P->kcap;
+  cp.topk = c.topk; cp.top_p = c.top_p; cp.kmin = c.kmin; cp.kmax = c.kmax;
+  cp.do_select = 0;
+  cp.scale = 1.0f / std::sqrt((float)D);
+  if (vsa::launch_coarse(cp, st) != cudaSuccess) return VSA_ERR_CUDA;
+
+  // 2. per-token preparation, transposed lists, coarse backward
+  if (!mark(1)) return VSA_ERR_CUDA;
+  vsa::PrepParams pp{};
+  pp.dout = static_cast<const __nv_bfloat16*>(dout);
+  pp.ofine = static_cast<const __nv_bfloat16*>(o_fine);
+  pp.lse = lse;
+  pp.gate_c = gate_c; pp.gate_f = gate_f;
+  pp.oc = cp.oc;
+  pp.do_cube = reinterpret_cast<__nv_bfloat16*>(bw + BL.do_cube);
+  pp.qstat = reinterpret_cast<float*>(bw + BL.qstat);
+  pp.doc = reinterpret_cast<float*>(bw + BL.doc);
+  pp.dlc = reinterpret_cast<float*>(bw + BL.dlc);
+  pp.dgate_c = dgate_c; pp.dgate_f = dgate_f;
+  pp.BH = P->BH; pp.C = P->C; pp.H = c.H; pp.W = c.W; pp.N = P->N;
+  if (vsa::launch_bwd_prep(pp, D, st) != cudaSuccess) return VSA_ERR_CUDA;
+  vsa::TlistParams tp{};
+  tp.idx = idx; tp.cnt = cnt;
+  tp.bitmap = reinterpret_cast<uint32_t*>(bw + BL.bitmap);
+  tp.tcnt = reinterpret_cast<int32_t*>(bw + BL.tcnt);
+  tp.toff = reinterpret_cast<int32_t*>(bw + BL.toff);
+  tp.tlist = reinterpret_cast<int32_t*>(bw + BL.tlist);
+  tp.err = cp.err;
+  tp.BH = P->BH; tp.C = P->C; tp.kcap = P->kcap; tp.W32 = (P->C + 31) / 32;
+  if (vsa::launch_tlists(tp, st) != cudaSuccess) return VSA_ERR_CUDA;
+  vsa::CoarseBwdParams cb{};
+  cb.psplit = cp.psplit; cb.Cp = cp.Cp;
+  cb.qbar = gp.pool[0]; cb.kbar = gp.pool[1]; cb.vbar = gp.pool[2];
+  cb.doc = pp.doc; cb.dlc = pp.dlc;
+  cb.p32 = reinterpret_cast<float*>(bw + BL.p32);
+  cb.ds = reinterpret_cast<float*>(bw + BL.ds);
+  cb.dqbar = reinterpret_cast<float*>(bw + BL.dqbar);
+  cb.dkbar = reinterpret_cast<float*>(bw + BL.dkbar);
+  cb.dvbar = reinterpret_cast<float*>(bw + BL.dvbar);
+  cb.BH = P->BH; cb.C = P->C; cb.D = D; cb.scale = cp.scale;
+  if (vsa::launch_coarse_bwd(cb, st) != cudaSuccess) return VSA_ERR_CUDA;
+
+  // 3. fine backward: dQ (query-major), then dK / dV (KV-major)
+  vsa::BwdFineParams fb{};
+  const size_t rows = (size_t)P->BH * P->N;
+  vsa_status e = VSA_OK;
+  fb.tm_q = P->tm_qc; fb.tm_k = P->tm_k; fb.tm_v = P->tm_v;
+  e = encode_cube_map(&fb.tm_do, bw + BL.do_cube, rows, D);
+  if (e == VSA_OK) e = encode_raster_map(&fb.tm_out0, dq, c, P->BH, false);
+  if (e != VSA_OK) return e;
+  fb.qstat = pp.qstat;
+  fb.err = cp.err;
+  fb.wait_ns = P->wait_ns;
+  fb.BH = P->BH; fb.C = P->C; fb.H = c.H; fb.W = c.W; fb.N = P->N; fb.kcap = P->kcap;
+  fb.n_items = P->BH * P->C;
+  fb.scale = cp.scale;
+  fb.scale_log2 = 1.4426950408889634f / std::sqrt((float)D);
+  fb.list = idx; fb.cnt = cnt; fb.off = nullptr;
+  fb.cpart0 = cb.dqbar; fb.cpart1 = nullptr;
+  const int grid = fb.n_items < P->num_sms ? fb.n_items : P->num_sms;
+  if (!mark(2)) return VSA_ERR_CUDA;
+  if (vsa::launch_fine_dq(fb, D, grid, st) != cudaSuccess) return VSA_ERR_CUDA;
+  e = encode_raster_map(&fb.tm_out0, dk, c, P->BH, false);
+  if (e == VSA_OK) e = encode_raster_map(&fb.tm_out1, dv, c, P->BH, false);
+  if (e != VSA_OK) return e;
+  fb.list = tp.tlist; fb.cnt = tp.tcnt; fb.off = tp.toff;
+  fb.cpart0 = cb.dkbar; fb.cpart1 = cb.dvbar;
+  if (!mark(3)) return VSA_ERR_CUDA;
+  if (vsa::launch_fine_dkv(fb, D, grid, st) != cudaSuccess) return VSA_ERR_CUDA;
+  if (!mark(4)) return VSA_ERR_CUDA;
+  if (timing) P->timed_bwd++;
   return VSA_OK;
 }
 
@@ -357,6 +524,7 @@ vsa_status vsa_plan(vsa_plan_t* out, const vsa_config* cfg, void* workspace, siz
   const size_t rows = (size_t)P->BH * P->N;
   vsa_status e = encode_cube_map(&P->tm_k, P->ws + L.k_cube, rows, cfg->D);
   if (e == VSA_OK) e = encode_cube_map(&P->tm_v, P->ws + L.v_cube, rows, cfg->D);
+  if (e == VSA_OK) e = encode_cube_map(&P->tm_qc, P->ws + L.q_cube, rows, cfg->D);
   if (e == VSA_OK) e = encode_coarse_maps(P);
   if (e == VSA_OK && cudaMemset(P->ws + L.err, 0, 16) != cudaSuccess) e = VSA_ERR_CUDA;
   if (e != VSA_OK) {
@@ -378,6 +546,37 @@ vsa_status vsa_run_fixed_idx(vsa_plan_t plan, const void* q, const void* k, cons
                              float* out_coarse, float* out_fine, void* stream) {
   return run_common(plan, q, k, v, gate_c, gate_f, false, idx_in, cnt_in, nullptr, nullptr, out, out_coarse, out_fine,
                     stream);
+}
+
+vsa_status vsa_run_train(vsa_plan_t plan, const void* q, const void* k, const void* v, const float* gate_c,
+                         const float* gate_f, void* out, int32_t* idx, int32_t* cnt, void* o_fine, float* lse,
+                         void* stream) {
+  if (!out || !o_fine || !lse) return VSA_ERR_INVALID_ARG;
+  return run_common(plan, q, k, v, gate_c, gate_f, true, nullptr, nullptr, idx, cnt, out, nullptr, nullptr, stream,
+                    o_fine, lse);
+}
+
+size_t vsa_backward_workspace_bytes(const vsa_config* cfg) {
+  if (validate(cfg) != VSA_OK) return 0;
+  BwdLayout L;
+  make_bwd_layout(cfg, &L);
+  return L.total;
+}
+
+vsa_status vsa_run_backward(vsa_plan_t plan, void* bwd_workspace, size_t bwd_bytes, const void* q, const void* k,
+                            const void* v, const float* gate_c, const float* gate_f, const int32_t* idx,
+                            const int32_t* cnt, const void* o_fine, const float* lse, const void* dout, void* dq,
+                            void* dk, void* dv, float* dgate_c, float* dgate_f, void* stream) {
+  return run_backward(plan, bwd_workspace, bwd_bytes, q, k, v, gate_c, gate_f, idx, cnt, o_fine, lse, dout, dq, dk,
+                      dv, dgate_c, dgate_f, stream);
+}
+
+vsa_status vsa_backward_stage_times(vsa_plan_t plan, float* ms) {
+  if (!plan || !ms || !plan->timing || plan->timed_bwd == 0) return VSA_ERR_INVALID_ARG;
+  if (cudaEventSynchronize(plan->evb[4]) != cudaSuccess) return VSA_ERR_CUDA;
+  for (int i = 0; i < 4; ++i)
+    if (cudaEventElapsedTime(&ms[i], plan->evb[i], plan->evb[i + 1]) != cudaSuccess) return VSA_ERR_CUDA;
+  return VSA_OK;
 }
 
 vsa_status vsa_run_host(vsa_plan_t plan, const void* q, const void* k, const void* v, const float* gate_c,
@@ -610,8 +809,12 @@ vsa_status vsa_check(vsa_plan_t plan) {
 
 void vsa_plan_destroy(vsa_plan_t plan) {
   if (!plan) return;
-  if (plan->ev[0])
-    for (int i = 0; i < 4; ++i) cudaEventDestroy(plan->ev[i]);
+  if (plan->ev) {
+    for (int i = 0; i < 4 * plan->ring; ++i) cudaEventDestroy(plan->ev[i]);
+    delete[] plan->ev;
+  }
+  if (plan->evb[0])
+    for (int i = 0; i < 5; ++i) cudaEventDestroy(plan->evb[i]);
   host_path_free(plan->host);
   delete plan;
 }
@@ -638,21 +841,52 @@ vsa_status vsa_set_wait_limit_ns(vsa_plan_t plan, uint64_t limit_ns) {
 
 vsa_status vsa_set_stage_timing(vsa_plan_t plan, int on) {
   if (!plan) return VSA_ERR_INVALID_ARG;
-  if (on && !plan->ev[0]) {
-    for (int i = 0; i < 4; ++i)
-      if (cudaEventCreate(&plan->ev[i]) != cudaSuccess) return VSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(plan->mu);
+  const int ring = on <= 0 ? 0 : (on > 4096 ? 4096 : on);
+  if (ring > plan->ring) {
+    cudaEvent_t* ev = new (std::nothrow) cudaEvent_t[4 * ring]();
+    if (!ev) return VSA_ERR_INVALID_ARG;
+    for (int i = 0; i < 4 * ring; ++i)
+      if (cudaEventCreate(&ev[i]) != cudaSuccess) {
+        for (int k = 0; k < i; ++k) cudaEventDestroy(ev[k]);
+        delete[] ev;
+        return VSA_ERR_CUDA;
+      }
+    if (plan->ev) {
+      for (int i = 0; i < 4 * plan->ring; ++i) cudaEventDestroy(plan->ev[i]);
+      delete[] plan->ev;
+    }
+    plan->ev = ev;
+    plan->ring = ring;
   }
-  plan->timing = on ? 1 : 0;
+  if (ring > 0 && !plan->evb[0]) {
+    for (int i = 0; i < 5; ++i)
+      if (cudaEventCreate(&plan->evb[i]) != cudaSuccess) return VSA_ERR_CUDA;
+  }
+  plan->timing = ring > 0 ? 1 : 0;
   plan->timed_runs = 0;
+  plan->timed_bwd = 0;
+  return VSA_OK;
+}
+
+vsa_status vsa_stage_times_history(vsa_plan_t plan, float* ms, int max_runs, int* n_runs) {
+  if (!plan || !ms || !n_runs || max_runs < 1 || !plan->timing || plan->timed_runs == 0) return VSA_ERR_INVALID_ARG;
+  const int kept = plan->timed_runs < plan->ring ? plan->timed_runs : plan->ring;
+  const int n = kept < max_runs ? kept : max_runs;
+  const int last = plan->timed_runs - 1;
+  if (cudaEventSynchronize(plan->ev[4 * (last % plan->ring) + 3]) != cudaSuccess) return VSA_ERR_CUDA;
+  for (int r = 0; r < n; ++r) {
+    const cudaEvent_t* e = plan->ev + 4 * ((last - (n - 1) + r) % plan->ring);
+    for (int i = 0; i < 3; ++i)
+      if (cudaEventElapsedTime(&ms[3 * r + i], e[i], e[i + 1]) != cudaSuccess) return VSA_ERR_CUDA;
+  }
+  *n_runs = n;
   return VSA_OK;
 }
 
 vsa_status vsa_stage_times(vsa_plan_t plan, float* ms) {
-  if (!plan || !ms || !plan->timing || plan->timed_runs == 0) return VSA_ERR_INVALID_ARG;
-  if (cudaEventSynchronize(plan->ev[3]) != cudaSuccess) return VSA_ERR_CUDA;
-  for (int i = 0; i < 3; ++i)
-    if (cudaEventElapsedTime(&ms[i], plan->ev[i], plan->ev[i + 1]) != cudaSuccess) return VSA_ERR_CUDA;
-  return VSA_OK;
+  int n = 0;
+  return vsa_stage_times_history(plan, ms, 1, &n);
 }
 
 int vsa_kernels_per_run(void) { return 5; }

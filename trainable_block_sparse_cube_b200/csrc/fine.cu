@@ -183,17 +183,6 @@ __device__ __forceinline__ void half_row_max(const uint32_t (&r)[32], float& x0,
   x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, 2));
 }
 
-// D[tmem] (+)= A[tmem] * B[smem]^T ; issued by a single thread.
-__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
-                                            uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 template <int D>
 struct Layout {
   static constexpr int NH = D / 64;              // 128-byte column groups of a row
@@ -232,6 +221,7 @@ struct alignas(16) Shared {
   int abort_flag;
   alignas(16) float xmax[2][64];      // [key half][row]: half-row maxima on the rescale path
   alignas(16) float lpart[2][2][64];  // [item parity][key half][row]: row sums of an item
+  alignas(16) float mref[2][64];      // [item parity][row]: final reference max (log2 units) of an item
   Pre pre[2];                         // [item parity]
 };
 
@@ -607,6 +597,10 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
       if ((lane & 3) == 0) {
         sh.lpart[ob][hf][ra] = l0;
         sh.lpart[ob][hf][ra + 8] = l1;
+        if (hf == 0) {
+          sh.mref[ob][ra] = m0;
+          sh.mref[ob][ra + 8] = m1;
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&B.l_full[ob]);
@@ -671,8 +665,16 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
       const int ob = is & 1;
       prefetch(is + 1);
       W.wait(&B.l_full[ob], (is >> 1) & 1);
-      const float il0 = 1.0f / (sh.lpart[ob][0][ra] + sh.lpart[ob][1][ra]);
-      const float il1 = 1.0f / (sh.lpart[ob][0][ra + 8] + sh.lpart[ob][1][ra + 8]);
+      const float lsum0 = sh.lpart[ob][0][ra] + sh.lpart[ob][1][ra];
+      const float lsum1 = sh.lpart[ob][0][ra + 8] + sh.lpart[ob][1][ra + 8];
+      const float il0 = 1.0f / lsum0, il1 = 1.0f / lsum1;
+      // raster token of in-cube slot q: ((4ct + q/16) H + 4ch + (q/4)%4) W + 4cw + q%4
+      auto tok_of = [&](int q) { return ((4 * ct + (q >> 4)) * p.H + 4 * ch + ((q >> 2) & 3)) * p.W + 4 * cw + (q & 3); };
+      if (p.lse && tq == 0) {
+        // natural log of the row's denominator: ln 2 * (reference max + log2 of the sum)
+        p.lse[(size_t)bh * p.N + tok_of(ra)] = 0.6931471805599453f * (sh.mref[ob][ra] + __log2f(lsum0));
+        p.lse[(size_t)bh * p.N + tok_of(ra + 8)] = 0.6931471805599453f * (sh.mref[ob][ra + 8] + __log2f(lsum1));
+      }
       W.wait(&B.o_full, is & 1);
       tc_fence_after();
       float o[2 * D / 4];
@@ -695,9 +697,18 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
       const Pre& pr = sh.pre[ob];
       const float gc0 = pr.gc[ra], gf0 = pr.gf[ra], gc1 = pr.gc[ra + 8], gf1 = pr.gf[ra + 8];
       // o[4j..4j+3] = (row ra: d, d+1; row ra+8: d, d+1), d = 8j + 2 tq
+      if (p.o_fine) {
+        const int tok0 = tok_of(ra), tok1 = tok_of(ra + 8);
+#pragma unroll
+        for (int jj = 0; jj < D / 8; ++jj) {
+          const int d = 8 * jj + 2 * tq;
+          *reinterpret_cast<__nv_bfloat162*>(p.o_fine + ((size_t)bh * p.N + tok0) * D + d) =
+              __floats2bfloat162_rn(o[4 * jj] * il0, o[4 * jj + 1] * il0);
+          *reinterpret_cast<__nv_bfloat162*>(p.o_fine + ((size_t)bh * p.N + tok1) * D + d) =
+              __floats2bfloat162_rn(o[4 * jj + 2] * il1, o[4 * jj + 3] * il1);
+        }
+      }
       if (p.out_fine) {
-        // raster token of in-cube slot q: ((4ct + q/16) H + 4ch + (q/4)%4) W + 4cw + q%4
-        auto tok_of = [&](int q) { return ((4 * ct + (q >> 4)) * p.H + 4 * ch + ((q >> 2) & 3)) * p.W + 4 * cw + (q & 3); };
         const int tok0 = tok_of(ra), tok1 = tok_of(ra + 8);
 #pragma unroll
         for (int jj = 0; jj < D / 8; ++jj) {

@@ -161,6 +161,58 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 }
 #undef VSA_R8
 
+// ---- 16-lane shapes (an M = 64 accumulator occupies lanes 0..15 of each
+// 32-lane quarter; these shapes spread those 16 lanes over a whole warp) ----
+#define VSA_O4(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3])
+#define VSA_I4(i) "r"(r[i]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3])
+// .16x256b.x4: 32 columns; r[4j..4j+3] = (row a: col c, c+1; row a+8: col c, c+1),
+// c = 8j + 2(t%4), a = t/4 (t = lane).
+__device__ __forceinline__ void tmem_ld16x256b_x4(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : VSA_O4(0), VSA_O4(4), VSA_O4(8), VSA_O4(12)
+      : "r"(taddr));
+}
+// .16x256b.x8: 64 columns, the same layout with j = 0..7.
+__device__ __forceinline__ void tmem_ld16x256b_x8(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x8.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : VSA_O4(0), VSA_O4(4), VSA_O4(8), VSA_O4(12), VSA_O4(16), VSA_O4(20), VSA_O4(24), VSA_O4(28)
+      : "r"(taddr));
+}
+// .16x128b.x4: 16 columns; r[2j] -> (row a, col 4j + t%4), r[2j+1] -> (row a+8, same col).
+__device__ __forceinline__ void tmem_st16x128b_x4(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.16x128b.x4.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), VSA_I4(0),
+               VSA_I4(4)
+               : "memory");
+}
+#undef VSA_O4
+#undef VSA_I4
+
+// D[tmem] (+)= A[tmem] * B[smem]^T ; issued by a single thread.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Untiled bulk copy global -> this CTA's shared memory, completing on an
+// mbarrier (transaction bytes). Both addresses 16-byte aligned, bytes a
+// multiple of 16.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // ---------------------------------------------------------------- tcgen05.mma
 // Shared-memory matrix descriptor, 128-byte swizzle.
 //   K-major operand: rows of 128 B (64 bf16 along K), 8-row groups SBO bytes

@@ -65,6 +65,8 @@ struct FineParams {
   const float* gate_f;           // [BH, N]
   __nv_bfloat16* out;            // [BH, N, D] or null
   float* out_fine;               // [BH, N, D] or null
+  __nv_bfloat16* o_fine;         // [BH, N, D] bf16 fine output saved for the backward pass, or null
+  float* lse;                    // [BH, N] natural-log softmax denominators saved for the backward pass, or null
   int* err;
   unsigned long long wait_ns;
   int BH, C, H, W, N, kcap, n_items;
@@ -72,9 +74,84 @@ struct FineParams {
   int debug_stall;
 };
 
+// ---------------------------------------------------------------- backward pass
+// Per-token preparation of the backward pass (one warp per query cube).
+struct PrepParams {
+  const __nv_bfloat16* dout;   // [BH, N, D] raster, gradient of the gated output
+  const __nv_bfloat16* ofine;  // [BH, N, D] raster, fine output saved by the forward
+  const float* lse;            // [BH, N] raster, natural-log softmax denominators saved by the forward
+  const float* gate_c;         // [BH, N]
+  const float* gate_f;         // [BH, N]
+  const float* oc;             // [BH, C, D] coarse output (recomputed)
+  __nv_bfloat16* do_cube;      // [BH, C, 64, D] gate_f * dout, cube-major (bf16)
+  float* qstat;                // [BH, C, 2, 64]: lse * log2(e) and delta = gate_f * (dout . ofine)
+  float* doc;                  // [BH, C, D] gradient of the coarse output
+  float* dlc;                  // [BH, C] doc . oc per cube
+  float* dgate_c;              // [BH, N]
+  float* dgate_f;              // [BH, N]
+  int BH, C, H, W, N;
+};
+
+// Backward of the coarse attention on the pooled tokens (fp32 SIMT products).
+struct CoarseBwdParams {
+  const __nv_bfloat16* psplit;  // [3, BH, C, Cp] coarse probabilities as three bf16 terms
+  int Cp;
+  const float* qbar;            // [BH, C, D] pooled q, k, v
+  const float* kbar;
+  const float* vbar;
+  const float* doc;             // [BH, C, D]
+  const float* dlc;             // [BH, C]
+  float* p32;                   // [BH, C, C] the probabilities in fp32
+  float* ds;                    // [BH, C, C] gradient of the coarse logits (unscaled)
+  float* dqbar;                 // [BH, C, D] gradients of the pooled q, k, v
+  float* dkbar;
+  float* dvbar;
+  int BH, C, D;
+  float scale;                  // 1/sqrt(D)
+};
+
+// Transposed selection lists: for every KV cube, the query cubes that selected it.
+struct TlistParams {
+  const int32_t* idx;   // [BH, C, kcap]
+  const int32_t* cnt;   // [BH, C] or null (every row holds kcap ids)
+  uint32_t* bitmap;     // [BH, C, W32] bit i of row j: query cube i selected KV cube j
+  int32_t* tcnt;        // [BH, C]
+  int32_t* toff;        // [BH, C] absolute offsets into tlist
+  int32_t* tlist;       // [BH * C * kcap] ascending query-cube ids per KV cube
+  int* err;
+  int BH, C, kcap, W32;
+};
+
+// Block-sparse fine attention backward (tcgen05). The dQ kernel walks query
+// cubes over their selected KV cubes; the dK/dV kernel walks KV cubes over
+// the query cubes that selected them.
+struct BwdFineParams {
+  // 2-D maps over cube-major copies [BH * C * 64][D] bf16, 64 x 64 boxes, 128-byte swizzle
+  CUtensorMap tm_q, tm_k, tm_v, tm_do;
+  // 5-D store maps over raster outputs [BH][T][H][W][D] bf16: dQ kernel tm_out0 = dq;
+  // dK/dV kernel tm_out0 = dk, tm_out1 = dv
+  CUtensorMap tm_out0, tm_out1;
+  const int32_t* list;   // dQ: idx [BH * C, kcap]; dK/dV: the flat transposed lists
+  const int32_t* cnt;    // dQ: counts or null (kcap each); dK/dV: tcnt
+  const int32_t* off;    // dK/dV: toff; dQ: null
+  const float* qstat;    // [BH * C, 2, 64]
+  const float* cpart0;   // [BH * C, D] coarse-path gradient rows: dQ kernel dq_bar; dK/dV kernel dk_bar
+  const float* cpart1;   // dK/dV kernel dv_bar
+  int* err;
+  unsigned long long wait_ns;
+  int BH, C, H, W, N, kcap, n_items;
+  float scale_log2;      // log2(e) / sqrt(D)
+  float scale;           // 1 / sqrt(D)
+};
+
 cudaError_t launch_gather(const GatherParams& p, int D, cudaStream_t st);
 cudaError_t launch_coarse(const CoarseParams& p, cudaStream_t st);
 cudaError_t launch_fine(const FineParams& p, int D, int grid, cudaStream_t st);
+cudaError_t launch_bwd_prep(const PrepParams& p, int D, cudaStream_t st);
+cudaError_t launch_coarse_bwd(const CoarseBwdParams& p, cudaStream_t st);
+cudaError_t launch_tlists(const TlistParams& p, cudaStream_t st);
+cudaError_t launch_fine_dq(const BwdFineParams& p, int D, int grid, cudaStream_t st);
+cudaError_t launch_fine_dkv(const BwdFineParams& p, int D, int grid, cudaStream_t st);
 cudaError_t launch_l2_read(const void* buf, size_t bytes, int passes, int* status, int grid, cudaStream_t st);
 
 }  // namespace vsa

@@ -39,7 +39,7 @@ import math
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "head_inputs", "make_inputs"]
+__all__ = ["Workload", "WORKLOADS", "head_inputs", "make_inputs", "head_dout", "make_dout"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -142,6 +142,19 @@ def head_inputs(wl: Workload, b: int, h: int):
     gate_f = torch.sigmoid(torch.randn(N, generator=g))
     bf = torch.bfloat16
     return q.to(bf), k.to(bf), v.to(bf), gate_c, gate_f
+
+
+def head_dout(wl: Workload, b: int, h: int) -> torch.Tensor:
+    """Upstream gradient of the gated output for one (b, head): [N, D] bf16,
+    N(0, 1) per element, from its own generator (seed offset so that it is
+    independent of the forward inputs)."""
+    g = torch.Generator().manual_seed(wl.seed * 1_000_003 + b * 1009 + h + 7_777_777)
+    return torch.randn(wl.N, wl.D, generator=g).to(torch.bfloat16)
+
+
+def make_dout(wl: Workload) -> torch.Tensor:
+    """Upstream gradients [B, heads, N, D] bf16 (see head_dout)."""
+    return torch.stack([torch.stack([head_dout(wl, b, h) for h in range(wl.heads)]) for b in range(wl.B)])
 
 
 def make_inputs(wl: Workload, heads=None):

@@ -21,7 +21,9 @@ STATUS = {0: "VSA_OK", 1: "VSA_ERR_INVALID_ARG", 2: "VSA_ERR_SHAPE", 3: "VSA_ERR
 EXPORTED = ["vsa_workspace_bytes", "vsa_workspace_layout", "vsa_plan", "vsa_run", "vsa_run_fixed_idx",
             "vsa_forward", "vsa_check", "vsa_plan_destroy", "vsa_status_string", "vsa_set_wait_limit_ns",
             "vsa_set_debug_stall", "vsa_set_stage_timing", "vsa_stage_times", "vsa_kernels_per_run",
-            "vsa_forward_noalloc", "vsa_set_cube_major_copies", "vsa_run_host", "vsa_measure_l2_read"]
+            "vsa_forward_noalloc", "vsa_set_cube_major_copies", "vsa_run_host", "vsa_measure_l2_read",
+            "vsa_run_train", "vsa_backward_workspace_bytes", "vsa_run_backward", "vsa_backward_stage_times",
+            "vsa_stage_times_history"]
 
 
 class VSAError(RuntimeError):
@@ -84,10 +86,20 @@ def load():
     L.vsa_set_stage_timing.restype = i32
     L.vsa_stage_times.argtypes = [vp, ctypes.POINTER(ctypes.c_float)]
     L.vsa_stage_times.restype = i32
+    L.vsa_stage_times_history.argtypes = [vp, ctypes.POINTER(ctypes.c_float), i32, ctypes.POINTER(ctypes.c_int)]
+    L.vsa_stage_times_history.restype = i32
     L.vsa_kernels_per_run.argtypes = []
     L.vsa_kernels_per_run.restype = i32
     L.vsa_forward_noalloc.argtypes = [vp] * 5 + [i32] * 7 + [ctypes.c_float, vp, vp, vp]
     L.vsa_forward_noalloc.restype = i32
+    L.vsa_run_train.argtypes = [vp] * 12
+    L.vsa_run_train.restype = i32
+    L.vsa_backward_workspace_bytes.argtypes = [ctypes.POINTER(Config)]
+    L.vsa_backward_workspace_bytes.restype = sz
+    L.vsa_run_backward.argtypes = [vp, vp, sz] + [vp] * 16
+    L.vsa_run_backward.restype = i32
+    L.vsa_backward_stage_times.argtypes = [vp, ctypes.POINTER(ctypes.c_float)]
+    L.vsa_backward_stage_times.restype = i32
     L.vsa_measure_l2_read.argtypes = [vp, sz, i32, vp, vp]
     L.vsa_measure_l2_read.restype = i32
     _lib = L
@@ -178,6 +190,50 @@ class Plan:
                               _ptr(cnt), _stream()), "vsa_run")
         return out, idx, cnt
 
+    def run_train(self, q, k, v, gate_c, gate_f):
+        """Forward pass that also saves the backward pass's inputs. Returns
+        (out, idx, cnt, o_fine, lse); enqueued on the current stream."""
+        self._inputs(q, k, v, gate_c, gate_f)
+        dev = q.device
+        out = torch.empty_like(q)
+        o_fine = torch.empty_like(q)
+        lse = torch.empty((self.B, self.heads, self.N), dtype=torch.float32, device=dev)
+        idx = torch.empty((self.B, self.heads, self.C, self.kcap), dtype=torch.int32, device=dev)
+        cnt = torch.empty((self.B, self.heads, self.C), dtype=torch.int32, device=dev)
+        _check(load().vsa_run_train(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(gate_c), _ptr(gate_f), _ptr(out),
+                                    _ptr(idx), _ptr(cnt), _ptr(o_fine), _ptr(lse), _stream()), "vsa_run_train")
+        return out, idx, cnt, o_fine, lse
+
+    def run_backward(self, q, k, v, gate_c, gate_f, idx, cnt, o_fine, lse, dout):
+        """Gradients of the gated output with the selection held fixed.
+        Returns (dq, dk, dv, dgate_c, dgate_f); enqueued on the current stream.
+        The backward workspace is allocated (once) by this plan."""
+        self._inputs(q, k, v, gate_c, gate_f)
+        BHND = (self.B, self.heads, self.N, self.D)
+        _need(idx, "idx", torch.int32, (self.B, self.heads, self.C, self.kcap))
+        if cnt is not None:
+            _need(cnt, "cnt", torch.int32, (self.B, self.heads, self.C))
+        _need(o_fine, "o_fine", torch.bfloat16, BHND)
+        _need(lse, "lse", torch.float32, BHND[:3])
+        _need(dout, "dout", torch.bfloat16, BHND)
+        L = load()
+        if getattr(self, "bwd_workspace", None) is None:
+            nb = L.vsa_backward_workspace_bytes(ctypes.byref(self.cfg))
+            self.bwd_workspace = torch.empty(nb, dtype=torch.uint8, device=q.device)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+        dgc, dgf = torch.empty_like(gate_c), torch.empty_like(gate_f)
+        _check(L.vsa_run_backward(self._h, _ptr(self.bwd_workspace), self.bwd_workspace.numel(), _ptr(q), _ptr(k),
+                                  _ptr(v), _ptr(gate_c), _ptr(gate_f), _ptr(idx), _ptr(cnt), _ptr(o_fine), _ptr(lse),
+                                  _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dgc), _ptr(dgf), _stream()),
+               "vsa_run_backward")
+        return dq, dk, dv, dgc, dgf
+
+    def backward_stage_times(self):
+        """Device ms of (gather + coarse, prep + lists + coarse backward, dq, dk/dv) of the last timed backward."""
+        ms = (ctypes.c_float * 4)()
+        _check(load().vsa_backward_stage_times(self._h, ms), "vsa_backward_stage_times")
+        return tuple(float(x) for x in ms)
+
     def run_host(self, q, k, v, gate_c, gate_f, out, idx, cnt=None):
         """Forward pass on host tensors (pinned for overlapped copies): inputs are
         copied in and out/idx/cnt written back by the library; enqueued on the
@@ -226,14 +282,24 @@ class Plan:
         """Also write the cube-major copy of q into the workspace (k and v are always copied)."""
         _check(load().vsa_set_cube_major_copies(self._h, 1 if on else 0), "vsa_set_cube_major_copies")
 
-    def set_stage_timing(self, on: bool):
-        _check(load().vsa_set_stage_timing(self._h, 1 if on else 0), "vsa_set_stage_timing")
+    def set_stage_timing(self, on):
+        """True (or a run count n >= 1): record stage events of the next runs,
+        keeping the last n (1 for True); False/0 switches timing off."""
+        n = int(on) if not isinstance(on, bool) else (1 if on else 0)
+        _check(load().vsa_set_stage_timing(self._h, n), "vsa_set_stage_timing")
 
     def stage_times(self):
         """Device ms of (gather+pool, coarse, fine) of the last timed run."""
         ms = (ctypes.c_float * 3)()
         _check(load().vsa_stage_times(self._h, ms), "vsa_stage_times")
         return tuple(float(x) for x in ms)
+
+    def stage_times_history(self, max_runs):
+        """[(gather+pool, coarse, fine) ms] of the last timed runs, oldest first."""
+        ms = (ctypes.c_float * (3 * max_runs))()
+        n = ctypes.c_int(0)
+        _check(load().vsa_stage_times_history(self._h, ms, int(max_runs), ctypes.byref(n)), "vsa_stage_times_history")
+        return [tuple(float(x) for x in ms[3 * i: 3 * i + 3]) for i in range(n.value)]
 
     # ------------------------------------------------------------ workspace views
     def workspace_view(self, region: str, dtype, shape):
