@@ -7,6 +7,7 @@ coarse attention + selection, fine attention + gated combine).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
   python bench.py --sweep [--steps K]        (one line per workload, with the oracle's CPU time)
+  python bench.py --backward [--workload W]  (one line for the backward pass)
   python bench.py --impl reference ...       (the fp64 CPU oracle, rank 0 only)
 
 Metric: sparse TFLOP/s of the forward pass, counting executed FLOPs only:
@@ -326,6 +327,83 @@ def run_sweep(args):
               f"{r['cpu_oracle']['s_per_call']:.1f} | {r['cpu_oracle']['cores']} |", file=sys.stderr)
 
 
+def run_backward_bench(args):
+    """One JSON line for the backward pass (vsa_run_backward) on the workload:
+    median device ms per call, its stage split, and per fine kernel the
+    executed tensor FLOPs over its event-timed duration against the measured
+    bf16 peak. Algorithmic FLOPs (the value): 2.5x the fine forward's (five
+    products per selected 64x64 block: S, dP, dV, dQ, dK) plus the coarse
+    backward's four C x C x D products per head. Executed in the kernels: dQ
+    three products per block (S, dP, dQ), dK/dV four (S^T, dP^T, dV, dK)."""
+    from trainable_block_sparse_cube_b200 import vsa
+
+    torch.cuda.set_device(0)
+    wl = synth.WORKLOADS[args.workload]
+    if args.heads:
+        wl = wl.with_(heads=args.heads)
+    q, k, v, gc, gf = synth.make_inputs(wl)
+    dev = tuple(t.cuda() for t in (q, k, v, gc, gf))
+    dout = synth.make_dout(wl).cuda()
+    plan = vsa.Plan(wl.B, wl.heads, wl.T, wl.H, wl.W, wl.D, wl.topk, wl.top_p, wl.kmin, wl.kmax)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    out, idx, cnt, of, lse = plan.run_train(*dev)
+    plan.check()
+    for _ in range(args.warmup):
+        plan.run_backward(*dev, idx, cnt, of, lse, dout)
+    plan.check()
+    f_fine, f_coarse = flops(wl, cnt.cpu().numpy())
+    sampler = ClockSampler(0)
+    sampler.start()
+    time.sleep(0.3)
+    plan.set_stage_timing(args.steps)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        plan.run_backward(*dev, idx, cnt, of, lse, dout)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    plan.check()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    st = np.median(np.array(plan.backward_stage_times_history(args.steps)), axis=0)
+    # the training forward, for reference (same timing scheme)
+    tf = []
+    for _ in range(max(5, args.steps // 4)):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        plan.run_train(*dev)
+        b.record(stream)
+        tf.append((a, b))
+    torch.cuda.synchronize()
+    train_ms = statistics.median(a.elapsed_time(b) for a, b in tf)
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    med = statistics.median(step_ms)
+    algo = 2.5 * f_fine + 2.0 * f_coarse
+    dq_t = 1.5 * f_fine / (st[2] * 1e-3) / 1e12
+    dkv_t = 2.0 * f_fine / (st[3] * 1e-3) / 1e12
+    line = {"metric": "VSA bwd ms/call & TFLOP/s (algorithmic) at the workload below", "value": algo / (med * 1e-3) / 1e12,
+            "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": med,
+            "ms_per_step_mean": float(np.mean(step_ms)), "higher_is_better": True, "dtype": "bf16",
+            "data": "synthetic", "config": {"workload": workload_desc(wl),
+                                             "l2": "256 MB L2 flush write between timed calls"},
+            "flops": {"algorithmic": algo, "fine_forward": f_fine, "coarse_forward": f_coarse},
+            "stages_ms": {"gather_coarse_recompute": float(st[0]), "prep_lists_coarse_bwd": float(st[1]),
+                          "fine_dq": float(st[2]), "fine_dkv": float(st[3])},
+            "roofline": {"bound": "tensor", "unit": "TFLOP/s", "peak": peak,
+                         "peak_source": f"{peak_src} bf16_tflops (burst)",
+                         "fine_dq_kernel": {"achieved": dq_t, "frac": dq_t / peak,
+                                            "executed_flops": 1.5 * f_fine},
+                         "fine_dkv_kernel": {"achieved": dkv_t, "frac": dkv_t / peak,
+                                             "executed_flops": 2.0 * f_fine}},
+            "train_forward_ms": train_ms,
+            "gpu_launches": 11 * args.steps, "clocks": clocks}
+    print(json.dumps(line), flush=True)
+
+
 def run_dry(args, rep):
     """Launcher self-test without a GPU: every rank times a small CPU step and
     the replica coordination (barrier, max over ranks, job throughput, one
@@ -493,6 +571,7 @@ def parse_args(argv=None):
     ap.add_argument("--sweep", action="store_true", help="one line per workload with the oracle's CPU time")
     ap.add_argument("--sweep-workloads", default="", help="comma-separated subset for --sweep")
     ap.add_argument("--dry-run", action="store_true", help="launcher self-test on CPU (gloo), no GPU work")
+    ap.add_argument("--backward", action="store_true", help="one line for the backward pass instead")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -504,6 +583,8 @@ def main():
     args = parse_args(argv)
     if args.sweep:
         return run_sweep(args)
+    if args.backward:
+        return run_backward_bench(args)
     env_world = os.environ.get("WORLD_SIZE")
     if env_world is not None:
         if int(env_world) != args.gpus and args.gpus != 1:

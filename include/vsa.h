@@ -134,8 +134,11 @@ vsa_status vsa_run_fixed_idx(vsa_plan_t plan, const void* q, const void* k, cons
  * "Approach": the hierarchy is trained end to end; "VSA: Faster Video
  * Diffusion with Trainable Sparse Attention", "Abstract (arXiv)": a single
  * differentiable kernel).
- *   o_fine: [B,heads,N,D] bf16, written: the fine-attention output before
- *           gating (raster order).
+ *   o_fine: [B,heads,N,D] fp32, written: the fine-attention output before
+ *           gating (raster order). fp32 because the backward pass forms
+ *           delta_n = dO_n . O_n from it: with O rounded to bf16 the error of
+ *           delta, multiplied by the softmax-weighted mean key in dq, can
+ *           exceed dq itself where attention is spread over similar keys.
  *   lse:    [B,heads,N] fp32, written: per token n, the natural log of its
  *           fine softmax denominator, log(sum_m exp(q_n . k_m / sqrt(D))) over
  *           the tokens m of its query cube's selected cubes (raster order).
@@ -288,8 +291,9 @@ vsa_status vsa_set_cube_major_copies(vsa_plan_t plan, int on);
 /* Stage timing for benchmarks. When `on` is positive, later runs of this plan
  * record CUDA events on the run's stream around its three stages: gather +
  * pool, coarse attention + selection, fine attention + combine; the events of
- * the last `on` runs are kept (at most 4096; created here). 0 switches timing
- * off. Every call restarts the count of recorded runs. */
+ * the last `on` runs are kept (at most 4096; created here), and likewise the
+ * four stages of vsa_run_backward calls. 0 switches timing off. Every call
+ * restarts the counts of recorded runs. */
 vsa_status vsa_set_stage_timing(vsa_plan_t plan, int on);
 
 /* Waits for the events of the last timed run and writes the device time of
@@ -308,6 +312,11 @@ vsa_status vsa_stage_times_history(vsa_plan_t plan, float* ms, int max_runs, int
  * backward, ms[2] fine dq, ms[3] fine dk / dv. VSA_ERR_INVALID_ARG if timing
  * is off or no backward ran since it was switched on. */
 vsa_status vsa_backward_stage_times(vsa_plan_t plan, float* ms);
+
+/* The backward stage times of the last min(max_runs, runs kept) timed
+ * vsa_run_backward calls, oldest first: ms[4 i + s] for call i and stage s
+ * (as in vsa_backward_stage_times); the count goes to *n_runs. */
+vsa_status vsa_backward_stage_times_history(vsa_plan_t plan, float* ms, int max_runs, int* n_runs);
 
 /* Number of kernel launches one vsa_run / vsa_run_fixed_idx call makes. */
 int vsa_kernels_per_run(void);

@@ -111,9 +111,31 @@ def assert_close(gpu, ref, what, max_abs=MAX_ABS, mean_abs=MEAN_ABS):
 # Gradients are compared relative to their own scale: with N(0, 1) upstream
 # gradients their magnitudes are ~1e-2, so the forward's absolute bounds would
 # pin nothing. The error is measured in units of the reference's RMS over the
-# compared elements.
-GRAD_MAX_REL = 3e-2
+# compared elements. The kernels round every product operand to bf16 (unit
+# roundoff u = 2^-8: dO, P and dS) and accumulate in fp32; the outputs are
+# bf16. A sum of bf16-rounded terms that partly cancel has an error of a few u
+# times the RMS of the result, and the largest of thousands of elements a few
+# times that: tests/test_backward_error_model.py replays those rounding steps
+# on the CPU and checks that these bounds sit between 1.5x and 8x the errors
+# the arithmetic produces.
+GRAD_MAX_REL = 0.15
 GRAD_MEAN_REL = 5e-3
+# The `cluster` inputs (tokens = one of 8 centres + 0.3 noise) make dq an
+# ill-conditioned sum: the selected keys of a query cube share one centre, the
+# softmax weights are near uniform, and dq = sum_m dS_m k_m cancels to a few
+# percent of its terms. An error e in delta_n = dO_n . O_n (O is computed
+# with bf16 P in the forward) enters dq as -e * (sum_m P_m k_m) / sqrt(D), on
+# the large common component of the keys, so the error floor of dq relative to
+# its own RMS is ~10x that of the other workloads (replayed on the CPU too).
+GRAD_ILL_DQ_MAX_REL = 1.5
+GRAD_ILL_DQ_MEAN_REL = 4e-2
+
+
+def grad_tolerance(wl, name):
+    """(max_rel, mean_rel) for gradient `name` of workload wl."""
+    if wl.gen == "cluster" and name == "dq":
+        return GRAD_ILL_DQ_MAX_REL, GRAD_ILL_DQ_MEAN_REL
+    return GRAD_MAX_REL, GRAD_MEAN_REL
 
 
 def assert_close_rel(gpu, ref, what, max_rel=GRAD_MAX_REL, mean_rel=GRAD_MEAN_REL):

@@ -14,7 +14,7 @@ import torch
 
 import oracle
 from oracle.vsa_oracle_backward import backward_head, fine_lse
-from parity import assert_close, assert_close_rel, oracle_head
+from parity import assert_close, assert_close_rel, grad_tolerance, oracle_head
 from test_gpu_parity import SMALL
 from trainable_block_sparse_cube_b200 import build as vsa_build
 from trainable_block_sparse_cube_b200 import synth, vsa
@@ -69,11 +69,8 @@ def test_backward_small(wl):
             assert_close(lse[b, h], lse_ref, "saved lse", max_abs=5e-4, mean_abs=5e-5)
             g = backward_head(_f64(q, b, h), _f64(k, b, h), _f64(v, b, h), _f64(gc, b, h), _f64(gf, b, h),
                               _f64(dout, b, h), wl.T, wl.H, wl.W, idx_h, cnt_h)
-            assert_close_rel(dq[b, h], g["dq"], f"{wl.name} dq")
-            assert_close_rel(dk[b, h], g["dk"], f"{wl.name} dk")
-            assert_close_rel(dv[b, h], g["dv"], f"{wl.name} dv")
-            assert_close_rel(dgc[b, h], g["dgate_c"], f"{wl.name} dgate_c")
-            assert_close_rel(dgf[b, h], g["dgate_f"], f"{wl.name} dgate_f")
+            for name, got in (("dq", dq), ("dk", dk), ("dv", dv), ("dgate_c", dgc), ("dgate_f", dgf)):
+                assert_close_rel(got[b, h], g[name], f"{wl.name} {name}", *grad_tolerance(wl, name))
 
 
 def test_backward_is_deterministic():
@@ -124,8 +121,11 @@ def test_backward_full_size_sampled(name):
     qt = np.concatenate([perm[64 * c: 64 * c + 64] for c in qc])
     kt = np.concatenate([perm[64 * c: 64 * c + 64] for c in kc])
     dq, dk, dv, dgc, dgf = grads
-    assert_close_rel(dq[0, h, torch.from_numpy(qt).cuda()].float().cpu().numpy(), g["dq"][qt], f"{name} dq")
-    assert_close_rel(dk[0, h, torch.from_numpy(kt).cuda()].float().cpu().numpy(), g["dk"][kt], f"{name} dk")
-    assert_close_rel(dv[0, h, torch.from_numpy(kt).cuda()].float().cpu().numpy(), g["dv"][kt], f"{name} dv")
-    assert_close_rel(dgc[0, h].cpu().numpy(), g["dgate_c"], f"{name} dgate_c")
-    assert_close_rel(dgf[0, h].cpu().numpy(), g["dgate_f"], f"{name} dgate_f")
+    assert_close_rel(dq[0, h, torch.from_numpy(qt).cuda()].float().cpu().numpy(), g["dq"][qt], f"{name} dq",
+                     *grad_tolerance(wl, "dq"))
+    assert_close_rel(dk[0, h, torch.from_numpy(kt).cuda()].float().cpu().numpy(), g["dk"][kt], f"{name} dk",
+                     *grad_tolerance(wl, "dk"))
+    assert_close_rel(dv[0, h, torch.from_numpy(kt).cuda()].float().cpu().numpy(), g["dv"][kt], f"{name} dv",
+                     *grad_tolerance(wl, "dv"))
+    assert_close_rel(dgc[0, h].cpu().numpy(), g["dgate_c"], f"{name} dgate_c", *grad_tolerance(wl, "dgate_c"))
+    assert_close_rel(dgf[0, h].cpu().numpy(), g["dgate_f"], f"{name} dgate_f", *grad_tolerance(wl, "dgate_f"))

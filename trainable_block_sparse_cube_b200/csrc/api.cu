@@ -54,7 +54,7 @@ struct vsa_plan_s {
   int timed_runs;    // runs recorded since timing was enabled
   cudaEvent_t* ev;     // stage events of the forward: 4 per run, for the last `ring` runs
   int ring;            // runs kept (vsa_set_stage_timing)
-  cudaEvent_t evb[5];  // backward stages: prologue, prep + lists + coarse, dQ, dK/dV
+  cudaEvent_t* evb;    // backward stage events: 5 per run (prologue, prep + lists + coarse, dQ, dK/dV), `ring` runs
   int timed_bwd;       // backward runs recorded since timing was enabled
   HostPath* host;    // vsa_run_host state (null until its first call)
 };
@@ -299,7 +299,7 @@ vsa_status run_common(vsa_plan_t P, const void* q, const void* k, const void* v,
   fp.gate_c = gate_c; fp.gate_f = gate_f;
   fp.out = static_cast<__nv_bfloat16*>(out);
   fp.out_fine = out_fine;
-  fp.o_fine = static_cast<__nv_bfloat16*>(o_fine);
+  fp.o_fine = static_cast<float*>(o_fine);
   fp.lse = lse;
   fp.err = reinterpret_cast<int*>(ws + L.err);
   fp.wait_ns = P->wait_ns;
@@ -348,8 +348,9 @@ vsa_status run_backward(vsa_plan_t P, void* bws, size_t bws_bytes, const void* q
   char* ws = P->ws;
   char* bw = static_cast<char*>(bws);
   const vsa_workspace_layout_t& L = P->lay;
-  const bool timing = P->timing && P->evb[0];
-  auto mark = [&](int i) { return !timing || cudaEventRecord(P->evb[i], st) == cudaSuccess; };
+  const bool timing = P->timing && P->evb;
+  cudaEvent_t* evb = timing ? P->evb + 5 * (P->timed_bwd % P->ring) : nullptr;
+  auto mark = [&](int i) { return !timing || cudaEventRecord(evb[i], st) == cudaSuccess; };
 
   // 1. gather + pool (with q's cube-major copy), coarse attention without selection
   if (!mark(0)) return VSA_ERR_CUDA;
@@ -386,7 +387,7 @@ vsa_status run_backward(vsa_plan_t P, void* bws, size_t bws_bytes, const void* q
   if (!mark(1)) return VSA_ERR_CUDA;
   vsa::PrepParams pp{};
   pp.dout = static_cast<const __nv_bfloat16*>(dout);
-  pp.ofine = static_cast<const __nv_bfloat16*>(o_fine);
+  pp.ofine = static_cast<const float*>(o_fine);
   pp.lse = lse;
   pp.gate_c = gate_c; pp.gate_f = gate_f;
   pp.oc = cp.oc;
@@ -571,12 +572,24 @@ vsa_status vsa_run_backward(vsa_plan_t plan, void* bwd_workspace, size_t bwd_byt
                       dv, dgate_c, dgate_f, stream);
 }
 
-vsa_status vsa_backward_stage_times(vsa_plan_t plan, float* ms) {
-  if (!plan || !ms || !plan->timing || plan->timed_bwd == 0) return VSA_ERR_INVALID_ARG;
-  if (cudaEventSynchronize(plan->evb[4]) != cudaSuccess) return VSA_ERR_CUDA;
-  for (int i = 0; i < 4; ++i)
-    if (cudaEventElapsedTime(&ms[i], plan->evb[i], plan->evb[i + 1]) != cudaSuccess) return VSA_ERR_CUDA;
+vsa_status vsa_backward_stage_times_history(vsa_plan_t plan, float* ms, int max_runs, int* n_runs) {
+  if (!plan || !ms || !n_runs || max_runs < 1 || !plan->timing || plan->timed_bwd == 0) return VSA_ERR_INVALID_ARG;
+  const int kept = plan->timed_bwd < plan->ring ? plan->timed_bwd : plan->ring;
+  const int n = kept < max_runs ? kept : max_runs;
+  const int last = plan->timed_bwd - 1;
+  if (cudaEventSynchronize(plan->evb[5 * (last % plan->ring) + 4]) != cudaSuccess) return VSA_ERR_CUDA;
+  for (int r = 0; r < n; ++r) {
+    const cudaEvent_t* e = plan->evb + 5 * ((last - (n - 1) + r) % plan->ring);
+    for (int i = 0; i < 4; ++i)
+      if (cudaEventElapsedTime(&ms[4 * r + i], e[i], e[i + 1]) != cudaSuccess) return VSA_ERR_CUDA;
+  }
+  *n_runs = n;
   return VSA_OK;
+}
+
+vsa_status vsa_backward_stage_times(vsa_plan_t plan, float* ms) {
+  int n = 0;
+  return vsa_backward_stage_times_history(plan, ms, 1, &n);
 }
 
 vsa_status vsa_run_host(vsa_plan_t plan, const void* q, const void* k, const void* v, const float* gate_c,
@@ -813,8 +826,10 @@ void vsa_plan_destroy(vsa_plan_t plan) {
     for (int i = 0; i < 4 * plan->ring; ++i) cudaEventDestroy(plan->ev[i]);
     delete[] plan->ev;
   }
-  if (plan->evb[0])
-    for (int i = 0; i < 5; ++i) cudaEventDestroy(plan->evb[i]);
+  if (plan->evb) {
+    for (int i = 0; i < 5 * plan->ring; ++i) cudaEventDestroy(plan->evb[i]);
+    delete[] plan->evb;
+  }
   host_path_free(plan->host);
   delete plan;
 }
@@ -852,16 +867,30 @@ vsa_status vsa_set_stage_timing(vsa_plan_t plan, int on) {
         delete[] ev;
         return VSA_ERR_CUDA;
       }
+    cudaEvent_t* evb = new (std::nothrow) cudaEvent_t[5 * ring]();
+    bool ok = evb != nullptr;
+    for (int i = 0; ok && i < 5 * ring; ++i)
+      if (cudaEventCreate(&evb[i]) != cudaSuccess) {
+        for (int k = 0; k < i; ++k) cudaEventDestroy(evb[k]);
+        ok = false;
+      }
+    if (!ok) {
+      for (int i = 0; i < 4 * ring; ++i) cudaEventDestroy(ev[i]);
+      delete[] ev;
+      delete[] evb;
+      return VSA_ERR_CUDA;
+    }
     if (plan->ev) {
       for (int i = 0; i < 4 * plan->ring; ++i) cudaEventDestroy(plan->ev[i]);
       delete[] plan->ev;
     }
+    if (plan->evb) {
+      for (int i = 0; i < 5 * plan->ring; ++i) cudaEventDestroy(plan->evb[i]);
+      delete[] plan->evb;
+    }
     plan->ev = ev;
+    plan->evb = evb;
     plan->ring = ring;
-  }
-  if (ring > 0 && !plan->evb[0]) {
-    for (int i = 0; i < 5; ++i)
-      if (cudaEventCreate(&plan->evb[i]) != cudaSuccess) return VSA_ERR_CUDA;
   }
   plan->timing = ring > 0 ? 1 : 0;
   plan->timed_runs = 0;

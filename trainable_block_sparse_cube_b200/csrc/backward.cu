@@ -11,7 +11,7 @@
 //   out_n = gc_n Oc[c(n)] + gf_n Of_n
 //   dgc_n = dout_n . Oc[c(n)],  dgf_n = dout_n . Of_n
 //   dOf_n = gf_n dout_n,        dOc[c] = sum over the cube's tokens of gc_n dout_n
-//   fine:   delta_n = dOf_n . Of_n = gf_n dgf_n; P = exp(s - lse); dS = P (dOf V^T - delta)
+//   fine:   delta_n = dOf_n . Of_n; P = exp(s - lse); dS = P (dOf V^T - delta)
 //   coarse: delta_c = dOc . Oc; dSc = Pc (dOc vbar^T - delta_c);
 //           dqbar = dSc kbar / sqrt(D), dkbar = dSc^T qbar / sqrt(D), dvbar = Pc^T dOc
 //   pool:   every token of cube c receives 1/64 of the pooled gradient.
@@ -55,21 +55,27 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const PrepParams p) {
     const int n = cube_token(c, r, p.H, p.W);
     const size_t row = (size_t)bh * p.N + n;
     const int4 dv = __ldg(reinterpret_cast<const int4*>(p.dout + row * D + chunk * 8));
-    const int4 ov = __ldg(reinterpret_cast<const int4*>(p.ofine + row * D + chunk * 8));
+    const float4 o_lo = __ldg(reinterpret_cast<const float4*>(p.ofine + row * D + chunk * 8));
+    const float4 o_hi = __ldg(reinterpret_cast<const float4*>(p.ofine + row * D + chunk * 8 + 4));
+    const float of[8] = {o_lo.x, o_lo.y, o_lo.z, o_lo.w, o_hi.x, o_hi.y, o_hi.z, o_hi.w};
     const float gc = __ldg(p.gate_c + row), gf = __ldg(p.gate_f + row);
     const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
-    const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
-    float pc = 0.f, pf = 0.f;
+    // pc = dout . Oc (dgate_c), pf = dout . Of (dgate_f), pd = bf16(gf dout) . Of: delta,
+    // formed from the same rounded dO the fine kernels' dP product uses, so that
+    // sum_m P_m (dP_m - delta) stays close to zero (it multiplies the
+    // P-weighted mean of the keys in dq).
+    float pc = 0.f, pf = 0.f, pd = 0.f;
     uint32_t w[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float2 d = __bfloat1622float2(d2[e]);
-      const float2 o = __bfloat1622float2(o2[e]);
       pc = fmaf(d.x, oc[2 * e], fmaf(d.y, oc[2 * e + 1], pc));
-      pf = fmaf(d.x, o.x, fmaf(d.y, o.y, pf));
+      pf = fmaf(d.x, of[2 * e], fmaf(d.y, of[2 * e + 1], pf));
       acc[2 * e] = fmaf(gc, d.x, acc[2 * e]);
       acc[2 * e + 1] = fmaf(gc, d.y, acc[2 * e + 1]);
       const __nv_bfloat162 g = __floats2bfloat162_rn(gf * d.x, gf * d.y);
+      const float2 gr = __bfloat1622float2(g);
+      pd = fmaf(gr.x, of[2 * e], fmaf(gr.y, of[2 * e + 1], pd));
       w[e] = *reinterpret_cast<const uint32_t*>(&g);
     }
     *reinterpret_cast<uint4*>(p.do_cube + (cube * kCube + r) * D + chunk * 8) = make_uint4(w[0], w[1], w[2], w[3]);
@@ -77,12 +83,13 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const PrepParams p) {
     for (int off = 1; off < LPR; off <<= 1) {
       pc += __shfl_xor_sync(0xffffffffu, pc, off);
       pf += __shfl_xor_sync(0xffffffffu, pf, off);
+      pd += __shfl_xor_sync(0xffffffffu, pd, off);
     }
     if (chunk == 0) {
       p.dgate_c[row] = pc;
       p.dgate_f[row] = pf;
       st[r] = __ldg(p.lse + row) * kLog2e;
-      st[64 + r] = gf * pf;
+      st[64 + r] = pd;
     }
   }
 #pragma unroll

@@ -702,10 +702,10 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
 #pragma unroll
         for (int jj = 0; jj < D / 8; ++jj) {
           const int d = 8 * jj + 2 * tq;
-          *reinterpret_cast<__nv_bfloat162*>(p.o_fine + ((size_t)bh * p.N + tok0) * D + d) =
-              __floats2bfloat162_rn(o[4 * jj] * il0, o[4 * jj + 1] * il0);
-          *reinterpret_cast<__nv_bfloat162*>(p.o_fine + ((size_t)bh * p.N + tok1) * D + d) =
-              __floats2bfloat162_rn(o[4 * jj + 2] * il1, o[4 * jj + 3] * il1);
+          *reinterpret_cast<float2*>(p.o_fine + ((size_t)bh * p.N + tok0) * D + d) =
+              make_float2(o[4 * jj] * il0, o[4 * jj + 1] * il0);
+          *reinterpret_cast<float2*>(p.o_fine + ((size_t)bh * p.N + tok1) * D + d) =
+              make_float2(o[4 * jj + 2] * il1, o[4 * jj + 3] * il1);
         }
       }
       if (p.out_fine) {

@@ -65,7 +65,7 @@ struct FineParams {
   const float* gate_f;           // [BH, N]
   __nv_bfloat16* out;            // [BH, N, D] or null
   float* out_fine;               // [BH, N, D] or null
-  __nv_bfloat16* o_fine;         // [BH, N, D] bf16 fine output saved for the backward pass, or null
+  float* o_fine;                 // [BH, N, D] fp32 fine output saved for the backward pass, or null
   float* lse;                    // [BH, N] natural-log softmax denominators saved for the backward pass, or null
   int* err;
   unsigned long long wait_ns;
@@ -78,13 +78,13 @@ struct FineParams {
 // Per-token preparation of the backward pass (one warp per query cube).
 struct PrepParams {
   const __nv_bfloat16* dout;   // [BH, N, D] raster, gradient of the gated output
-  const __nv_bfloat16* ofine;  // [BH, N, D] raster, fine output saved by the forward
+  const float* ofine;          // [BH, N, D] raster, fp32 fine output saved by the forward
   const float* lse;            // [BH, N] raster, natural-log softmax denominators saved by the forward
   const float* gate_c;         // [BH, N]
   const float* gate_f;         // [BH, N]
   const float* oc;             // [BH, C, D] coarse output (recomputed)
   __nv_bfloat16* do_cube;      // [BH, C, 64, D] gate_f * dout, cube-major (bf16)
-  float* qstat;                // [BH, C, 2, 64]: lse * log2(e) and delta = gate_f * (dout . ofine)
+  float* qstat;                // [BH, C, 2, 64]: lse * log2(e) and delta = bf16(gate_f dout) . ofine
   float* doc;                  // [BH, C, D] gradient of the coarse output
   float* dlc;                  // [BH, C] doc . oc per cube
   float* dgate_c;              // [BH, N]

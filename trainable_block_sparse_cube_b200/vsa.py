@@ -23,7 +23,7 @@ EXPORTED = ["vsa_workspace_bytes", "vsa_workspace_layout", "vsa_plan", "vsa_run"
             "vsa_set_debug_stall", "vsa_set_stage_timing", "vsa_stage_times", "vsa_kernels_per_run",
             "vsa_forward_noalloc", "vsa_set_cube_major_copies", "vsa_run_host", "vsa_measure_l2_read",
             "vsa_run_train", "vsa_backward_workspace_bytes", "vsa_run_backward", "vsa_backward_stage_times",
-            "vsa_stage_times_history"]
+            "vsa_stage_times_history", "vsa_backward_stage_times_history"]
 
 
 class VSAError(RuntimeError):
@@ -100,6 +100,8 @@ def load():
     L.vsa_run_backward.restype = i32
     L.vsa_backward_stage_times.argtypes = [vp, ctypes.POINTER(ctypes.c_float)]
     L.vsa_backward_stage_times.restype = i32
+    L.vsa_backward_stage_times_history.argtypes = [vp, ctypes.POINTER(ctypes.c_float), i32, ctypes.POINTER(ctypes.c_int)]
+    L.vsa_backward_stage_times_history.restype = i32
     L.vsa_measure_l2_read.argtypes = [vp, sz, i32, vp, vp]
     L.vsa_measure_l2_read.restype = i32
     _lib = L
@@ -196,7 +198,7 @@ class Plan:
         self._inputs(q, k, v, gate_c, gate_f)
         dev = q.device
         out = torch.empty_like(q)
-        o_fine = torch.empty_like(q)
+        o_fine = torch.empty(q.shape, dtype=torch.float32, device=dev)
         lse = torch.empty((self.B, self.heads, self.N), dtype=torch.float32, device=dev)
         idx = torch.empty((self.B, self.heads, self.C, self.kcap), dtype=torch.int32, device=dev)
         cnt = torch.empty((self.B, self.heads, self.C), dtype=torch.int32, device=dev)
@@ -213,7 +215,7 @@ class Plan:
         _need(idx, "idx", torch.int32, (self.B, self.heads, self.C, self.kcap))
         if cnt is not None:
             _need(cnt, "cnt", torch.int32, (self.B, self.heads, self.C))
-        _need(o_fine, "o_fine", torch.bfloat16, BHND)
+        _need(o_fine, "o_fine", torch.float32, BHND)
         _need(lse, "lse", torch.float32, BHND[:3])
         _need(dout, "dout", torch.bfloat16, BHND)
         L = load()
@@ -227,6 +229,14 @@ class Plan:
                                   _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dgc), _ptr(dgf), _stream()),
                "vsa_run_backward")
         return dq, dk, dv, dgc, dgf
+
+    def backward_stage_times_history(self, max_runs):
+        """[(gather + coarse, prep + lists + coarse backward, dq, dk/dv) ms] of the last timed backward calls."""
+        ms = (ctypes.c_float * (4 * max_runs))()
+        n = ctypes.c_int(0)
+        _check(load().vsa_backward_stage_times_history(self._h, ms, int(max_runs), ctypes.byref(n)),
+               "vsa_backward_stage_times_history")
+        return [tuple(float(x) for x in ms[4 * i: 4 * i + 4]) for i in range(n.value)]
 
     def backward_stage_times(self):
         """Device ms of (gather + coarse, prep + lists + coarse backward, dq, dk/dv) of the last timed backward."""
