@@ -135,7 +135,7 @@ void make_layout(const vsa_config* c, vsa_workspace_layout_t* L, bool with_q_cub
 
 // Regions of the backward pass's workspace (byte offsets).
 struct BwdLayout {
-  size_t do_cube, qstat, doc, dlc, p32, ds, dqbar, dkbar, dvbar, bitmap, tcnt, toff, tlist, total;
+  size_t do_cube, qstat, doc, docsplit, dlc, dssplit, dqbar, dkbar, dvbar, bitmap, tcnt, toff, tlist, total;
 };
 void make_bwd_layout(const vsa_config* c, BwdLayout* L) {
   const size_t BH = (size_t)c->B * c->heads, N = (size_t)c->T * c->H * c->W, C = N / 64, D = c->D;
@@ -149,9 +149,9 @@ void make_bwd_layout(const vsa_config* c, BwdLayout* L) {
   L->do_cube = take(BH * N * D * 2);
   L->qstat = take(BH * C * 128 * 4);
   L->doc = take(BH * C * D * 4);
+  L->docsplit = take(3 * BH * C * D * 2);
   L->dlc = take(BH * C * 4);
-  L->p32 = take(BH * C * C * 4);
-  L->ds = take(BH * C * C * 4);
+  L->dssplit = take(3 * BH * C * coarse_pitch(C) * 2);
   L->dqbar = take(BH * C * D * 4);
   L->dkbar = take(BH * C * D * 4);
   L->dvbar = take(BH * C * D * 4);
@@ -394,6 +394,7 @@ vsa_status run_backward(vsa_plan_t P, void* bws, size_t bws_bytes, const void* q
   pp.do_cube = reinterpret_cast<__nv_bfloat16*>(bw + BL.do_cube);
   pp.qstat = reinterpret_cast<float*>(bw + BL.qstat);
   pp.doc = reinterpret_cast<float*>(bw + BL.doc);
+  pp.docsplit = reinterpret_cast<__nv_bfloat16*>(bw + BL.docsplit);
   pp.dlc = reinterpret_cast<float*>(bw + BL.dlc);
   pp.dgate_c = dgate_c; pp.dgate_f = dgate_f;
   pp.BH = P->BH; pp.C = P->C; pp.H = c.H; pp.W = c.W; pp.N = P->N;
@@ -408,14 +409,30 @@ vsa_status run_backward(vsa_plan_t P, void* bws, size_t bws_bytes, const void* q
   tp.BH = P->BH; tp.C = P->C; tp.kcap = P->kcap; tp.W32 = (P->C + 31) / 32;
   if (vsa::launch_tlists(tp, st) != cudaSuccess) return VSA_ERR_CUDA;
   vsa::CoarseBwdParams cb{};
-  cb.psplit = cp.psplit; cb.Cp = cp.Cp;
-  cb.qbar = gp.pool[0]; cb.kbar = gp.pool[1]; cb.vbar = gp.pool[2];
-  cb.doc = pp.doc; cb.dlc = pp.dlc;
-  cb.p32 = reinterpret_cast<float*>(bw + BL.p32);
-  cb.ds = reinterpret_cast<float*>(bw + BL.ds);
+  {
+    const size_t BHs = P->BH, Cs = P->C, Ds = D, Cp = coarse_pitch(Cs), tbytes = 3 * BHs * Cs * Ds * 2;
+    char* pool = ws + L.pool_split;  // [q, k, v][3 terms][BH][C][D]
+    char* docs = bw + BL.docsplit;
+    char* dss = bw + BL.dssplit;
+    vsa_status me = encode_planes_map(&cb.tm_doc128, docs, Ds, Ds, Cs, 3 * BHs, 128);
+    if (me == VSA_OK) me = encode_planes_map(&cb.tm_vb128, pool + 2 * tbytes, Ds, Ds, Cs, 3 * BHs, 128);
+    if (me == VSA_OK) me = encode_planes_map(&cb.tm_ds128, dss, Cp, Cp, Cs, 3 * BHs, 128);
+    if (me == VSA_OK) me = encode_planes_map(&cb.tm_kb64, pool + tbytes, Ds, Ds, Cs, 3 * BHs, 64);
+    if (me == VSA_OK) me = encode_planes_map(&cb.tm_qb64, pool, Ds, Ds, Cs, 3 * BHs, 64);
+    if (me == VSA_OK) me = encode_planes_map(&cb.tm_doc64, docs, Ds, Ds, Cs, 3 * BHs, 64);
+    if (me == VSA_OK) me = encode_planes_map(&cb.tm_ds64, dss, Cp, Cp, Cs, 3 * BHs, 64);
+    if (me == VSA_OK) me = encode_planes_map(&cb.tm_p64, ws + L.p_split, Cp, Cp, Cs, 3 * BHs, 64);
+    if (me != VSA_OK) return me;
+  }
+  cb.psplit = cp.psplit;
+  cb.dssplit = reinterpret_cast<__nv_bfloat16*>(bw + BL.dssplit);
+  cb.Cp = cp.Cp;
+  cb.dlc = pp.dlc;
   cb.dqbar = reinterpret_cast<float*>(bw + BL.dqbar);
   cb.dkbar = reinterpret_cast<float*>(bw + BL.dkbar);
   cb.dvbar = reinterpret_cast<float*>(bw + BL.dvbar);
+  cb.err = cp.err;
+  cb.wait_ns = P->wait_ns;
   cb.BH = P->BH; cb.C = P->C; cb.D = D; cb.scale = cp.scale;
   if (vsa::launch_coarse_bwd(cb, st) != cudaSuccess) return VSA_ERR_CUDA;
 

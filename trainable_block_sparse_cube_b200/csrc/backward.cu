@@ -14,7 +14,9 @@
 //   fine:   delta_n = dOf_n . Of_n; P = exp(s - lse); dS = P (dOf V^T - delta)
 //   coarse: delta_c = dOc . Oc; dSc = Pc (dOc vbar^T - delta_c);
 //           dqbar = dSc kbar / sqrt(D), dkbar = dSc^T qbar / sqrt(D), dvbar = Pc^T dOc
+//           (tensor cores, fp32-accurate three-term bf16 operands)
 //   pool:   every token of cube c receives 1/64 of the pooled gradient.
+#include "sm100_ptx.cuh"
 #include "vsa_common.cuh"
 
 namespace vsa {
@@ -106,125 +108,257 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const PrepParams p) {
     d4[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
     d4[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
     if (chunk == 0) p.dlc[cube] = dl;
+    // dOc as three bf16 terms for the tensor-core coarse backward
+    uint32_t w[3][4];
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+      float x[2] = {acc[e], acc[e + 1]};
+#pragma unroll
+      for (int t = 0; t < 3; ++t) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(x[0], x[1]);
+        const float2 back = __bfloat1622float2(h);
+        x[0] -= back.x;
+        x[1] -= back.y;
+        w[t][e / 2] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+    }
+    const size_t plane = (size_t)p.BH * p.C * D;
+#pragma unroll
+    for (int t = 0; t < 3; ++t)
+      *reinterpret_cast<uint4*>(p.docsplit + t * plane + cube * D + chunk * 8) = make_uint4(w[t][0], w[t][1], w[t][2], w[t][3]);
   }
 }
 
 // ------------------------------------------------------------ coarse backward
-// fp32 SIMT products on 64 x 64 output tiles (16-deep k chunks in shared
-// memory, 4 x 4 outputs per thread). The coarse stage is C x C per head, a few
-// percent of the backward pass's work.
-constexpr int kT = 64, kKc = 16;
+// Four products per head on the tensor cores (tcgen05, M = 128, fp32 in TMEM),
+// every fp32 operand as three bf16 terms x = hi + mid + lo and the six
+// products hi.hi, hi.mid, mid.hi, mid.mid, hi.lo, lo.hi summed (the dropped
+// ones are below 2^-24 relative), so the products keep fp32 accuracy: dS
+// feeds sums that cancel (sum_j dS_ij = 0), like the fine path's.
+//   KIND 0: dPc = dOc vbar^T   [C x C], K = D; epilogue dS = Pc (dPc - delta_c) as three terms
+//   KIND 1: dqbar = dS kbar / sqrt(D)    [C x D], K = C (A = dS, K-major)
+//   KIND 2: dkbar = dS^T qbar / sqrt(D)  [C x D], K = C (A = dS^T, MN-major loads of dS)
+//   KIND 3: dvbar = Pc^T dOc             [C x D], K = C (A = Pc^T, MN-major loads of Pc)
+// One CTA per 128-row tile: warp 0 issues the TMA loads (all three terms of
+// A and B for 64 of K per stage), warp 1 the 6 x 4 MMAs of a stage, all four
+// warps read the accumulator. Every wait is bounded (records kErrTimeout).
+template <int KIND, int D>
+struct BwTc {
+  static constexpr int NT = KIND == 0 ? 128 : D;
+  static constexpr int A_BYTES = 128 * 64 * 2;
+  static constexpr int B_BYTES = NT * 64 * 2;
+  static constexpr int STAGE = 3 * (A_BYTES + B_BYTES);
+  static constexpr int NS = KIND == 0 ? 1 : 2;
+  static constexpr int SMEM = NS * STAGE + 1024;
+};
 
-// dSc = Pc (dOc vbar^T - delta_c); also writes Pc in fp32 for the dvbar product.
-__global__ void __launch_bounds__(256) coarse_ds_kernel(const CoarseBwdParams p) {
-  __shared__ float As[kKc][kT + 4], Bs[kKc][kT + 4];
-  const int tid = threadIdx.x, tm = tid >> 4, tn = tid & 15;
-  const int m0 = blockIdx.x * kT, n0 = blockIdx.y * kT, bh = blockIdx.z;
-  const int C = p.C, D = p.D;
-  const float* A = p.doc + (size_t)bh * C * D;    // [C][D]: A(m, k) = doc[m][k]
-  const float* B = p.vbar + (size_t)bh * C * D;   // B(k, n) = vbar[n][k]
-  float acc[4][4] = {};
-  for (int k0 = 0; k0 < D; k0 += kKc) {
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int idx = tid + 256 * e;
-      const int m = idx >> 4, kk = idx & 15;
-      As[kk][m] = (m0 + m < C) ? A[(size_t)(m0 + m) * D + k0 + kk] : 0.f;
-      Bs[kk][m] = (n0 + m < C) ? B[(size_t)(n0 + m) * D + k0 + kk] : 0.f;
+__device__ __forceinline__ void split3(float x, __nv_bfloat16& h, __nv_bfloat16& m, __nv_bfloat16& l) {
+  h = __float2bfloat16_rn(x);
+  const float r1 = x - __bfloat162float(h);
+  m = __float2bfloat16_rn(r1);
+  l = __float2bfloat16_rn(r1 - __bfloat162float(m));
+}
+
+template <int KIND, int D>
+__global__ void __launch_bounds__(128, KIND == 0 ? 2 : 1)
+    coarse_bwd_tc_kernel(const __grid_constant__ CoarseBwdParams p) {
+  using S = BwTc<KIND, D>;
+  using namespace ptx;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t full[2], empty[2], done;
+  __shared__ uint32_t tmem_base;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int C = p.C, BH = p.BH;
+  const int m0 = blockIdx.x * 128, n0 = blockIdx.y * S::NT, bh = blockIdx.z;
+  const int K = KIND == 0 ? D : (KIND == 1 ? p.Cp : C);
+  const int nch = (K + 63) / 64;
+  const uint64_t lim = p.wait_ns;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
     }
-    __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < kKc; ++kk) {
-      float a[4], b[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        a[i] = As[kk][tm * 4 + i];
-        b[i] = Bs[kk][tn * 4 + i];
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
-    }
-    __syncthreads();
+    mbar_init(&done, 1);
+    fence_mbar_init();
   }
-  const size_t plane = (size_t)p.BH * C * p.Cp;
+  if (warp == 0) {
+    tmem_alloc(&tmem_base, S::NT);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+  auto a_tile = [&](int st, int t) { return tiles + st * S::STAGE + t * S::A_BYTES; };
+  auto b_tile = [&](int st, int t) { return tiles + st * S::STAGE + 3 * S::A_BYTES + t * S::B_BYTES; };
+
+  if (warp == 0 && lane == 0) {
+    int armed = 0;
+    for (int c = 0; c < nch; ++c) {
+      const int st = c % S::NS;
+      if (c >= S::NS && !mbar_wait(&empty[st], ((c / S::NS) - 1) & 1, lim)) {
+        atomicOr(p.err, kErrTimeout);
+        break;
+      }
+      mbar_arrive_expect_tx(&full[st], S::STAGE);
+      ++armed;
+      for (int t = 0; t < 3; ++t) {
+        const int plane = t * BH + bh;
+        if (KIND == 0) {
+          tma_load_3d(a_tile(st, t), &p.tm_doc128, &full[st], 64 * c, m0, plane);
+          tma_load_3d(b_tile(st, t), &p.tm_vb128, &full[st], 64 * c, n0, plane);
+        } else {
+          if (KIND == 1) {
+            tma_load_3d(a_tile(st, t), &p.tm_ds128, &full[st], 64 * c, m0, plane);
+          } else {
+            const CUtensorMap* ta = KIND == 2 ? &p.tm_ds64 : &p.tm_p64;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int m = m0 + tm * 4 + i;
-    if (m >= C) continue;
-    const float dl = p.dlc[(size_t)bh * C + m];
-    const __nv_bfloat16* prow = p.psplit + ((size_t)bh * C + m) * p.Cp;
+            for (int mh = 0; mh < 2; ++mh) tma_load_3d(a_tile(st, t) + mh * 8192, ta, &full[st], m0 + 64 * mh, 64 * c, plane);
+          }
+          const CUtensorMap* tb = KIND == 1 ? &p.tm_kb64 : (KIND == 2 ? &p.tm_qb64 : &p.tm_doc64);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int n = n0 + tn * 4 + j;
-      if (n >= C) continue;
-      const float P = __bfloat162float(prow[n]) + __bfloat162float(prow[plane + n]) +
-                      __bfloat162float(prow[2 * plane + n]);
-      const size_t o = ((size_t)bh * C + m) * C + n;
-      p.p32[o] = P;
-      p.ds[o] = P * (acc[i][j] - dl);
+          for (int h = 0; h < D / 64; ++h) tma_load_3d(b_tile(st, t) + h * 8192, tb, &full[st], 64 * h, 64 * c, plane);
+        }
+      }
     }
+    for (int st = 0; st < S::NS && st < armed; ++st) mbar_wait(&full[st], ((armed - 1 - st) / S::NS) & 1, lim);
+  } else if (warp == 1 && lane == 0) {
+    constexpr uint32_t idesc = idesc_bf16_f32(128, S::NT, KIND >= 2, KIND >= 1);
+    constexpr int pa[6] = {2, 0, 1, 1, 0, 0}, pb[6] = {0, 2, 1, 0, 1, 0};
+    bool ok = true;
+    for (int c = 0; c < nch && ok; ++c) {
+      const int st = c % S::NS;
+      if (!mbar_wait(&full[st], (c / S::NS) & 1, lim)) {
+        atomicOr(p.err, kErrTimeout);
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+        for (int q = 0; q < 6; ++q) {
+          uint64_t ad, bd;
+          if (KIND >= 2) ad = sdesc_sw128(smem_u32(a_tile(st, pa[q])), 8192, 1024) + (uint64_t)((kk * 2048) >> 4);
+          else ad = sdesc_sw128(smem_u32(a_tile(st, pa[q])), 16, 1024) + (uint64_t)((kk * 32) >> 4);
+          if (KIND == 0) bd = sdesc_sw128(smem_u32(b_tile(st, pb[q])), 16, 1024) + (uint64_t)((kk * 32) >> 4);
+          else bd = sdesc_sw128(smem_u32(b_tile(st, pb[q])), 8192, 1024) + (uint64_t)((kk * 2048) >> 4);
+          mma_bf16_ss(tmem, ad, bd, idesc, (c > 0 || kk > 0 || q > 0) ? 1u : 0u);
+        }
+      mma_commit(&empty[st]);
+    }
+    mma_commit(&done);
+  }
+  __syncwarp();
+  const bool have = mbar_wait(&done, 0, lim);
+  if (!have && lane == 0) atomicOr(p.err, kErrTimeout);
+  tc_fence_after();
+  const int row = m0 + 32 * warp + lane;
+  const size_t cp_plane = (size_t)BH * C * p.Cp;
+#pragma unroll 1
+  for (int cg = 0; cg < S::NT / 32; ++cg) {
+    uint32_t r[32];
+    tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16) + 32 * cg, r);
+    tmem_wait_ld();
+    if (!have || row >= C) continue;
+    if (KIND == 0) {
+      const int j0 = n0 + 32 * cg;
+      if (j0 >= p.Cp) continue;
+      const float dl = p.dlc[(size_t)bh * C + row];
+      const size_t o = ((size_t)bh * C + row) * p.Cp + j0;
+      if (j0 + 32 <= C) {
+        // 32 columns of the row: 16-byte loads of the three P terms and 16-byte
+        // stores of the three dS terms (row pitch Cp * 2 bytes, a multiple of 16)
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4) {
+          uint4 pt[3];
+#pragma unroll
+          for (int t = 0; t < 3; ++t) pt[t] = *reinterpret_cast<const uint4*>(p.psplit + t * cp_plane + o + 8 * v4);
+          uint32_t w[3][4];
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            float ds[2];
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int e = 8 * v4 + 2 * e2 + h2;
+              float P = 0.f;
+#pragma unroll
+              for (int t = 0; t < 3; ++t) {
+                const uint32_t word = (&pt[t].x)[e2];
+                P += __uint_as_float((h2 ? (word & 0xffff0000u) : (word << 16)));
+              }
+              ds[h2] = P * (__uint_as_float(r[e]) - dl);
+            }
+            float x[2] = {ds[0], ds[1]};
+#pragma unroll
+            for (int t = 0; t < 3; ++t) {
+              const __nv_bfloat162 hh = __floats2bfloat162_rn(x[0], x[1]);
+              const float2 back = __bfloat1622float2(hh);
+              x[0] -= back.x;
+              x[1] -= back.y;
+              w[t][e2] = *reinterpret_cast<const uint32_t*>(&hh);
+            }
+          }
+#pragma unroll
+          for (int t = 0; t < 3; ++t)
+            *reinterpret_cast<uint4*>(p.dssplit + t * cp_plane + o + 8 * v4) = make_uint4(w[t][0], w[t][1], w[t][2], w[t][3]);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int j = j0 + e;
+          if (j >= p.Cp) continue;
+          float ds = 0.f;
+          if (j < C) {
+            const float P = __bfloat162float(p.psplit[o + e]) + __bfloat162float(p.psplit[cp_plane + o + e]) +
+                            __bfloat162float(p.psplit[2 * cp_plane + o + e]);
+            ds = P * (__uint_as_float(r[e]) - dl);
+          }
+          __nv_bfloat16 h, m, l;
+          split3(ds, h, m, l);
+          p.dssplit[o + e] = h;
+          p.dssplit[cp_plane + o + e] = m;
+          p.dssplit[2 * cp_plane + o + e] = l;
+        }
+      }
+    } else {
+      float* out = KIND == 1 ? p.dqbar : (KIND == 2 ? p.dkbar : p.dvbar);
+      const float alpha = KIND == 3 ? 1.0f : p.scale;
+      const size_t o = ((size_t)bh * C + row) * D + 32 * cg;
+#pragma unroll
+      for (int e = 0; e < 32; e += 4)
+        *reinterpret_cast<float4*>(out + o + e) =
+            make_float4(alpha * __uint_as_float(r[e]), alpha * __uint_as_float(r[e + 1]),
+                        alpha * __uint_as_float(r[e + 2]), alpha * __uint_as_float(r[e + 3]));
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, S::NT);
   }
 }
 
-// out[m][d] = alpha * sum_k A(m, k) * B[k][d] with M = K = C and N = D:
-//   z = 0: dvbar = Pc^T dOc             (A(m, k) = p32[k][m])
-//   z = 1: dqbar = dSc kbar / sqrt(D)   (A(m, k) = ds[m][k])
-//   z = 2: dkbar = dSc^T qbar / sqrt(D) (A(m, k) = ds[k][m])
-__global__ void __launch_bounds__(256) coarse_grad_kernel(const CoarseBwdParams p) {
-  __shared__ float As[kKc][kT + 4], Bs[kKc][kT + 4];
-  const int tid = threadIdx.x, tm = tid >> 4, tn = tid & 15;
-  const int m0 = blockIdx.x * kT, n0 = blockIdx.y * kT;
-  const int which = blockIdx.z % 3, bh = blockIdx.z / 3;
-  const int C = p.C, D = p.D;
-  const size_t cc = (size_t)bh * C * C, cd = (size_t)bh * C * D;
-  const float* A = which == 0 ? p.p32 + cc : p.ds + cc;
-  const bool at = which != 1;
-  const float* B = (which == 0 ? p.doc : which == 1 ? p.kbar : p.qbar) + cd;
-  float* out = (which == 0 ? p.dvbar : which == 1 ? p.dqbar : p.dkbar) + cd;
-  const float alpha = which == 0 ? 1.f : p.scale;
-  float acc[4][4] = {};
-  for (int k0 = 0; k0 < C; k0 += kKc) {
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int idx = tid + 256 * e;
-      if (at) {
-        const int m = idx & 63, kk = idx >> 6;
-        As[kk][m] = (m0 + m < C && k0 + kk < C) ? A[(size_t)(k0 + kk) * C + m0 + m] : 0.f;
-      } else {
-        const int m = idx >> 4, kk = idx & 15;
-        As[kk][m] = (m0 + m < C && k0 + kk < C) ? A[(size_t)(m0 + m) * C + k0 + kk] : 0.f;
-      }
-      const int n = idx & 63, kk = idx >> 6;
-      Bs[kk][n] = (k0 + kk < C && n0 + n < D) ? B[(size_t)(k0 + kk) * D + n0 + n] : 0.f;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < kKc; ++kk) {
-      float a[4], b[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        a[i] = As[kk][tm * 4 + i];
-        b[i] = Bs[kk][tn * 4 + i];
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int m = m0 + tm * 4 + i;
-    if (m >= C) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int n = n0 + tn * 4 + j;
-      if (n < D) out[(size_t)m * D + n] = alpha * acc[i][j];
-    }
-  }
+template <int KIND, int D>
+cudaError_t launch_bw_tc(const CoarseBwdParams& p, cudaStream_t st) {
+  using S = BwTc<KIND, D>;
+  cudaError_t e =
+      cudaFuncSetAttribute(coarse_bwd_tc_kernel<KIND, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((p.C + 127) / 128, KIND == 0 ? (p.Cp + 127) / 128 : 1, p.BH);
+  coarse_bwd_tc_kernel<KIND, D><<<grid, 128, S::SMEM, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_coarse_bwd_t(const CoarseBwdParams& p, cudaStream_t st) {
+  cudaError_t e = launch_bw_tc<0, D>(p, st);
+  if (e == cudaSuccess) e = launch_bw_tc<1, D>(p, st);
+  if (e == cudaSuccess) e = launch_bw_tc<2, D>(p, st);
+  if (e == cudaSuccess) e = launch_bw_tc<3, D>(p, st);
+  return e;
 }
 
 // ------------------------------------------------------------ transposed lists
@@ -318,12 +452,7 @@ cudaError_t launch_bwd_prep(const PrepParams& p, int D, cudaStream_t st) {
 }
 
 cudaError_t launch_coarse_bwd(const CoarseBwdParams& p, cudaStream_t st) {
-  const int tc = (p.C + kT - 1) / kT;
-  coarse_ds_kernel<<<dim3(tc, tc, p.BH), 256, 0, st>>>(p);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  coarse_grad_kernel<<<dim3(tc, (p.D + kT - 1) / kT, 3 * p.BH), 256, 0, st>>>(p);
-  return cudaGetLastError();
+  return p.D == 128 ? launch_coarse_bwd_t<128>(p, st) : launch_coarse_bwd_t<64>(p, st);
 }
 
 cudaError_t launch_tlists(const TlistParams& p, cudaStream_t st) {

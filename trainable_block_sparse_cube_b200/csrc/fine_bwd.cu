@@ -22,18 +22,19 @@
 // accumulators use the M=64 TMEM layout (16 lanes of each 32-lane quarter);
 // the softmax-side warps read and write them with the 16-lane shapes.
 //
-// bf16 packing into TMEM: a softmax warp handles 32 of a step's 64 columns
-// (half h) and writes its 16 packed bf16-pair columns at column 32h of the
-// same buffer, inside the range it alone reads, so the two warps of a lane
-// quarter never overwrite each other's unread fp32 values. The MMA that reads
-// them takes its K = 16 slices at packed columns {0, 8, 32, 40}.
+// The eight elementwise warps form two groups that take alternate steps
+// (group g: the steps j with j % 2 == g), so the TMEM round trips of two
+// steps overlap; a warp handles all 64 columns of its lane quarter and writes
+// its 32 packed bf16-pair columns over the first 32 fp32 columns it has
+// already read (no other warp reads that quarter of the buffer). The MMA that
+// reads them takes its K = 16 slices at packed columns 8k.
 //
 // Warp roles (512 threads), both kernels:
 //   warp 0      TMA producer (tiles and the per-query statistics)
 //   warp 1      issuer of the S (or S^T) MMAs; allocates tensor memory
 //   warp 2      issuer of the dP (or dP^T) MMAs
 //   warp 3      issuer of the accumulating MMAs (dQ; or dV and dK)
-//   warps 4-11  elementwise: P, dS (warp w: lane quarter w % 4, column half (w-4)/4)
+//   warps 4-11  elementwise: P, dS (warp w: lane quarter w % 4, step parity (w-4)/4)
 //   warps 12-15 epilogue: accumulators -> scale, add the coarse path's
 //               gradient / 64, bf16, 5-D TMA store into the raster output
 // Every mbarrier wait is bounded (the plan's wait limit); a wait that gives
@@ -64,7 +65,7 @@ template <int N>
 __device__ __forceinline__ void regs_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
 
 // Packed bf16 column of K = 16 slice k of a 64-column step (see the header).
-__device__ __forceinline__ uint32_t packed_col(int k) { return (k < 2) ? 8u * k : 32u + 8u * (k - 2); }
+__device__ __forceinline__ uint32_t packed_col(int k) { return 8u * k; }
 
 // K-major operand slice k (16 elements along D) of a 64-row tile laid out as
 // D/64 blocks of [64 rows][128 B] in the 128-byte swizzle: descriptor offset.
@@ -174,15 +175,15 @@ __device__ __forceinline__ void load_acc(uint32_t taddr, float* o) {
 }
 
 // Elementwise step of the softmax warps: s (scores) and g (dP) of rows a and
-// a+8 for 32 columns (layout of tmem_ld16x256b_x4); lse2 and delta per row
+// a+8 for 64 columns (layout of tmem_ld16x256b_x8); lse2 and delta per row
 // (dQ kernel: ROWSTAT) or per column (dK/dV kernel). Writes P (packed bf16
-// pairs) to pk_p and dS to pk_s.
+// pairs) to pk_p and dS to pk_s (layout of the 16x128b.x8 store).
 template <bool ROWSTAT>
-__device__ __forceinline__ void p_ds(const uint32_t (&s)[16], const uint32_t (&g)[16], float sl2, float l0, float l1,
+__device__ __forceinline__ void p_ds(const uint32_t (&s)[32], const uint32_t (&g)[32], float sl2, float l0, float l1,
                                      float d0, float d1, const float* lse_col, const float* dl_col, int c0,
-                                     uint32_t (&pk_p)[8], uint32_t (&pk_s)[8]) {
+                                     uint32_t (&pk_p)[16], uint32_t (&pk_s)[16]) {
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
+  for (int j = 0; j < 8; ++j) {
     float la0 = l0, la1 = l0, lb0 = l1, lb1 = l1, da0 = d0, da1 = d0, db0 = d1, db1 = d1;
     if (!ROWSTAT) {
       const int c = c0 + 8 * j;
@@ -230,7 +231,7 @@ constexpr int kNb = 3;  // S / dP buffers in the dQ kernel
 constexpr uint32_t kQS = 0, kQP = 192, kQAcc = 384;
 
 struct __align__(8) DqBars {
-  uint64_t k_full[4], k_empty[4], v_full[3], v_empty[3];
+  uint64_t k_full[8], k_empty[8], v_full[8], v_empty[8];  // rings of DqL<D>::KS / VS slots
   uint64_t q_full[2], q_empty[2];
   uint64_t s_full[kNb], dp_full[kNb], ds_full[kNb], dp_free[kNb], sp_free[kNb];
   uint64_t acc_full, acc_empty;
@@ -261,8 +262,8 @@ __global__ void __launch_bounds__(kThreads, 1) fine_dq_kernel(const __grid_const
     for (int b = 0; b < kNb; ++b) {
       mbar_init(&B.s_full[b], 1);
       mbar_init(&B.dp_full[b], 1);
-      mbar_init(&B.ds_full[b], 8);
-      mbar_init(&B.dp_free[b], 8);
+      mbar_init(&B.ds_full[b], 4);
+      mbar_init(&B.dp_free[b], 4);
       mbar_init(&B.sp_free[b], 1);
     }
     mbar_init(&B.acc_full, 1);
@@ -296,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1) fine_dq_kernel(const __grid_const
       Cur c;
       cur_init<false>(p, c);
       while (c.live && !aborted) {
-        const int bh = c.item / C, ci = c.item - bh * C;
+        const int bh = c.item / C;
         // Q, dO and the statistics of the item -> buffer is & 1.
         const int qb = c.is & 1;
         if (c.is >= 2 && !W.wait(&B.q_empty[qb], ((c.is >> 1) - 1) & 1)) { aborted = true; break; }
@@ -421,11 +422,11 @@ __global__ void __launch_bounds__(kThreads, 1) fine_dq_kernel(const __grid_const
     __syncwarp();
   } else if (warp < 12) {
     // ------------------------------------------------------------ P, dS
-    const int quarter = warp & 3, hf = (warp - 4) >> 2;
+    const int quarter = warp & 3, grp = (warp - 4) >> 2;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const int ra = quarter * 16 + (lane >> 2);
     const float sl2 = p.scale_log2;
-    int b = 0, u = 0;
+    int j = 0, b = 0, u = 0;  // CTA step, its S/dP buffer and use count
     Cur c;
     cur_init<false>(p, c);
     while (c.live) {
@@ -436,23 +437,26 @@ __global__ void __launch_bounds__(kThreads, 1) fine_dq_kernel(const __grid_const
       __syncwarp();
       if (lane == 0) mbar_arrive(&B.q_empty[qb]);
       for (int t = 0; t < c.n; ++t) {
-        W.wait(&B.s_full[b], u & 1);
-        W.wait(&B.dp_full[b], u & 1);
-        tc_fence_after();
-        uint32_t s[16], g[16];
-        tmem_ld16x256b_x4(tmem + lane_base + kQS + 64u * b + 32u * hf, s);
-        tmem_ld16x256b_x4(tmem + lane_base + kQP + 64u * b + 32u * hf, g);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&B.dp_free[b]);
-        uint32_t pk_p[8], pk_s[8];
-        p_ds<true>(s, g, sl2, l0, l1, d0, d1, nullptr, nullptr, 0, pk_p, pk_s);
-        tmem_st16x128b_x4(tmem + lane_base + kQS + 64u * b + 32u * hf, pk_s);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&B.ds_full[b]);
+        if ((j & 1) == grp) {
+          W.wait(&B.s_full[b], u & 1);
+          W.wait(&B.dp_full[b], u & 1);
+          tc_fence_after();
+          uint32_t sr[32], g[32];
+          tmem_ld16x256b_x8(tmem + lane_base + kQS + 64u * b, sr);
+          tmem_ld16x256b_x8(tmem + lane_base + kQP + 64u * b, g);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&B.dp_free[b]);
+          uint32_t pk_p[16], pk_s[16];
+          p_ds<true>(sr, g, sl2, l0, l1, d0, d1, nullptr, nullptr, 0, pk_p, pk_s);
+          tmem_st16x128b_x8(tmem + lane_base + kQS + 64u * b, pk_s);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&B.ds_full[b]);
+        }
+        ++j;
         if (++b == kNb) { b = 0; ++u; }
       }
       cur_next_item<false>(p, c);
@@ -550,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1) fine_dkv_kernel(const __grid_cons
     for (int b = 0; b < kNt; ++b) {
       mbar_init(&B.st_full[b], 1);
       mbar_init(&B.dpt_full[b], 1);
-      mbar_init(&B.pt_full[b], 8);
+      mbar_init(&B.pt_full[b], 4);
       mbar_init(&B.st_free[b], 1);
     }
     mbar_init(&B.acc_full, 1);
@@ -718,33 +722,36 @@ __global__ void __launch_bounds__(kThreads, 1) fine_dkv_kernel(const __grid_cons
     __syncwarp();
   } else if (warp < 12) {
     // ------------------------------------------------------------ P^T, dS^T
-    const int quarter = warp & 3, hf = (warp - 4) >> 2;
+    // Two S^T / dP^T buffers and two groups: group g always works on buffer g.
+    const int quarter = warp & 3, grp = (warp - 4) >> 2;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    const int c0 = 32 * hf + 2 * (lane & 3);  // first query column of the thread (plus 8 j)
+    const int c0 = 2 * (lane & 3);  // first query column of the thread (plus 8 j)
     const float sl2 = p.scale_log2;
     int g = 0, b = 0, u = 0;
     Cur c;
     cur_init<true>(p, c);
     while (c.live) {
       for (int t = 0; t < c.n; ++t) {
-        const int rs = g % L::RS;
-        W.wait(&B.r_full[rs], (g / L::RS) & 1);
-        W.wait(&B.st_full[b], u & 1);
-        W.wait(&B.dpt_full[b], u & 1);
-        tc_fence_after();
-        const float* stat = reinterpret_cast<const float*>(tiles + L::OFF_RING + rs * L::SLOT + 2 * L::TILE);
-        uint32_t s[16], gg[16];
-        tmem_ld16x256b_x4(tmem + lane_base + kTS + 64u * b + 32u * hf, s);
-        tmem_ld16x256b_x4(tmem + lane_base + kTP + 64u * b + 32u * hf, gg);
-        tmem_wait_ld();
-        uint32_t pk_p[8], pk_s[8];
-        p_ds<false>(s, gg, sl2, 0.f, 0.f, 0.f, 0.f, stat, stat + 64, c0, pk_p, pk_s);
-        tmem_st16x128b_x4(tmem + lane_base + kTS + 64u * b + 32u * hf, pk_p);
-        tmem_st16x128b_x4(tmem + lane_base + kTP + 64u * b + 32u * hf, pk_s);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&B.pt_full[b]);
+        if (b == grp) {
+          const int rs = g % L::RS;
+          W.wait(&B.r_full[rs], (g / L::RS) & 1);
+          W.wait(&B.st_full[b], u & 1);
+          W.wait(&B.dpt_full[b], u & 1);
+          tc_fence_after();
+          const float* stat = reinterpret_cast<const float*>(tiles + L::OFF_RING + rs * L::SLOT + 2 * L::TILE);
+          uint32_t s[32], gg[32];
+          tmem_ld16x256b_x8(tmem + lane_base + kTS + 64u * b, s);
+          tmem_ld16x256b_x8(tmem + lane_base + kTP + 64u * b, gg);
+          tmem_wait_ld();
+          uint32_t pk_p[16], pk_s[16];
+          p_ds<false>(s, gg, sl2, 0.f, 0.f, 0.f, 0.f, stat, stat + 64, c0, pk_p, pk_s);
+          tmem_st16x128b_x8(tmem + lane_base + kTS + 64u * b, pk_p);
+          tmem_st16x128b_x8(tmem + lane_base + kTP + 64u * b, pk_s);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&B.pt_full[b]);
+        }
         ++g;
         if (++b == kNt) { b = 0; ++u; }
       }

@@ -189,6 +189,14 @@ __device__ __forceinline__ void tmem_st16x128b_x4(uint32_t taddr, const uint32_t
                VSA_I4(4)
                : "memory");
 }
+// .16x128b.x8: 32 columns; r[2j] -> (row a, col 4j + t%4), r[2j+1] -> (row a+8, same col).
+__device__ __forceinline__ void tmem_st16x128b_x8(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x128b.x8.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      VSA_I4(0), VSA_I4(4), VSA_I4(8), VSA_I4(12)
+      : "memory");
+}
 #undef VSA_O4
 #undef VSA_I4
 

@@ -86,26 +86,31 @@ struct PrepParams {
   __nv_bfloat16* do_cube;      // [BH, C, 64, D] gate_f * dout, cube-major (bf16)
   float* qstat;                // [BH, C, 2, 64]: lse * log2(e) and delta = bf16(gate_f dout) . ofine
   float* doc;                  // [BH, C, D] gradient of the coarse output
+  __nv_bfloat16* docsplit;     // [3, BH, C, D] the same as three bf16 terms (hi, mid, lo)
   float* dlc;                  // [BH, C] doc . oc per cube
   float* dgate_c;              // [BH, N]
   float* dgate_f;              // [BH, N]
   int BH, C, H, W, N;
 };
 
-// Backward of the coarse attention on the pooled tokens (fp32 SIMT products).
+// Backward of the coarse attention on the pooled tokens: four C x C x D
+// products per head on the tensor cores, each fp32 operand as three bf16
+// terms (as in the forward's coarse products).
 struct CoarseBwdParams {
-  const __nv_bfloat16* psplit;  // [3, BH, C, Cp] coarse probabilities as three bf16 terms
+  // 3-D maps [3 * BH][rows][cols] over three-term bf16 operands, 128-byte swizzle, boxes {64 cols, rows}:
+  CUtensorMap tm_doc128, tm_vb128;         // dOc, vbar [C][D], 128-row boxes (dS product: A, B K-major)
+  CUtensorMap tm_ds128;                    // dS [C][Cp], 128-row boxes (dqbar product: A K-major)
+  CUtensorMap tm_kb64, tm_qb64, tm_doc64;  // kbar, qbar, dOc [C][D], 64-row boxes (B operands, N-major)
+  CUtensorMap tm_ds64, tm_p64;             // dS, P [C][Cp], 64-row boxes (A MN-major: dkbar, dvbar products)
+  const __nv_bfloat16* psplit;  // [3, BH, C, Cp] coarse probabilities (three terms), read by the dS epilogue
+  __nv_bfloat16* dssplit;       // [3, BH, C, Cp] dS = P (dOc vbar^T - delta_c) as three terms (written)
   int Cp;
-  const float* qbar;            // [BH, C, D] pooled q, k, v
-  const float* kbar;
-  const float* vbar;
-  const float* doc;             // [BH, C, D]
   const float* dlc;             // [BH, C]
-  float* p32;                   // [BH, C, C] the probabilities in fp32
-  float* ds;                    // [BH, C, C] gradient of the coarse logits (unscaled)
   float* dqbar;                 // [BH, C, D] gradients of the pooled q, k, v
   float* dkbar;
   float* dvbar;
+  int* err;
+  unsigned long long wait_ns;
   int BH, C, D;
   float scale;                  // 1/sqrt(D)
 };
