@@ -95,6 +95,9 @@ typedef struct {
                                     probabilities as three bf16 terms, Cp = C
                                     rounded up to a multiple of 8 (zero padded)   */
   size_t cnt;                    /* [B*heads, C] int32 counts used by the fine step */
+  size_t order;                  /* [B*heads*C] int32 work order of the fine step
+                                    when counts vary (each head's query cubes
+                                    longest first)                              */
   size_t err;                    /* int32 device error word                        */
   size_t total;                  /* == vsa_workspace_bytes                          */
 } vsa_workspace_layout_t;
@@ -318,7 +321,9 @@ vsa_status vsa_backward_stage_times(vsa_plan_t plan, float* ms);
  * (as in vsa_backward_stage_times); the count goes to *n_runs. */
 vsa_status vsa_backward_stage_times_history(vsa_plan_t plan, float* ms, int max_runs, int* n_runs);
 
-/* Number of kernel launches one vsa_run / vsa_run_fixed_idx call makes. */
+/* Number of kernel launches one vsa_run / vsa_run_fixed_idx call makes in
+ * top-K mode (5). With variable counts (top-p, or vsa_run_fixed_idx given
+ * counts) one more kernel orders the fine step's work longest first. */
 int vsa_kernels_per_run(void);
 
 /* Measurement hook (not a step of the method; the pages have no counterpart):

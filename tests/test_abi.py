@@ -78,9 +78,19 @@ def test_layout_sizes(lib):
     assert lay.total == lib.vsa_workspace_bytes(ctypes.byref(c))
     assert lay.p_split - lay.pool_split >= 9 * BH * C * D * 2
     assert lay.cnt - lay.p_split >= 3 * BH * C * ((C + 7) // 8 * 8) * 2
+    assert lay.err - lay.order >= BH * C * 4
     offs = [lay.q_cube, lay.k_cube, lay.v_cube, lay.q_pool, lay.k_pool, lay.v_pool, lay.o_coarse, lay.s_coarse,
-            lay.pool_split, lay.p_split, lay.cnt, lay.err]
+            lay.pool_split, lay.p_split, lay.cnt, lay.order, lay.err]
     assert offs == sorted(offs) and all(o % 1024 == 0 for o in offs)
+
+
+def test_backward_workspace_size(lib):
+    c = _cfg(B=1, heads=2, T=8, H=12, W=16, D=128, topk=5)
+    BH, N, C, D = 2, 8 * 12 * 16, 8 * 12 * 16 // 64, 128
+    nb = lib.vsa_backward_workspace_bytes(ctypes.byref(c))
+    # at least: dO cube-major, statistics, dOc (+ terms), dS terms, pooled gradients, lists, orders
+    assert nb >= BH * N * D * 2 + BH * C * 128 * 4 + BH * C * D * (4 + 6) + 3 * BH * C * ((C + 7) // 8 * 8) * 2
+    assert lib.vsa_backward_workspace_bytes(ctypes.byref(_cfg(B=1, heads=2, T=6, H=12, W=16, D=128, topk=5))) == 0
 
 
 def test_plan_argument_errors(lib):

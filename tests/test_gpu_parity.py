@@ -293,3 +293,19 @@ def test_maximum_cube_count(mode):
     toks = np.concatenate([r["perm"][64 * c: 64 * c + 64] for c in cubes])
     got = out[0, 0, torch.from_numpy(toks).cuda()].float().cpu().numpy()
     assert_close(got, r["out"][toks], f"{mode} sampled output")
+
+
+def test_work_order_is_longest_first_per_head():
+    """With variable counts the fine step's items are handed out from an order
+    array: each head's query cubes by descending count, ties by ascending id,
+    heads in sequence (a permutation of all items)."""
+    wl = SMALL[4]                                   # top-p, variable counts
+    plan, dev_in, out, idx, cnt = _run(wl, synth.make_inputs(wl))
+    BH = wl.B * wl.heads
+    order = plan.workspace_view("order", torch.int32, (BH * wl.C,)).cpu().numpy()
+    counts = cnt.cpu().numpy().reshape(BH, wl.C)
+    assert sorted(order.tolist()) == list(range(BH * wl.C))
+    for bh in range(BH):
+        ids = np.arange(wl.C)
+        want = bh * wl.C + ids[np.lexsort((ids, -counts[bh]))]
+        assert np.array_equal(order[bh * wl.C:(bh + 1) * wl.C], want)

@@ -9,7 +9,7 @@ import subprocess
 import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-SRC = ["api.cu", "gather.cu", "coarse.cu", "fine.cu", "measure.cu", "backward.cu", "fine_bwd.cu"]
+SRC = ["api.cu", "gather.cu", "coarse.cu", "fine.cu", "measure.cu", "backward.cu", "fine_bwd.cu", "schedule.cu"]
 LIB = os.path.join(HERE, "libvsa.so")
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

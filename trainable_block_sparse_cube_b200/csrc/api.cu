@@ -129,13 +129,15 @@ void make_layout(const vsa_config* c, vsa_workspace_layout_t* L, bool with_q_cub
   L->pool_split = take(9 * BH * C * D * 2);
   L->p_split = take(3 * BH * C * coarse_pitch(C) * 2);
   L->cnt = take(BH * C * 4);
+  L->order = take(BH * C * 4);
   L->err = take(16);
   L->total = off;
 }
 
 // Regions of the backward pass's workspace (byte offsets).
 struct BwdLayout {
-  size_t do_cube, qstat, doc, docsplit, dlc, dssplit, dqbar, dkbar, dvbar, bitmap, tcnt, toff, tlist, total;
+  size_t do_cube, qstat, doc, docsplit, dlc, dssplit, dqbar, dkbar, dvbar, bitmap, tcnt, toff, tlist, order_q,
+      order_kv, total;
 };
 void make_bwd_layout(const vsa_config* c, BwdLayout* L) {
   const size_t BH = (size_t)c->B * c->heads, N = (size_t)c->T * c->H * c->W, C = N / 64, D = c->D;
@@ -159,6 +161,8 @@ void make_bwd_layout(const vsa_config* c, BwdLayout* L) {
   L->tcnt = take(BH * C * 4);
   L->toff = take(BH * C * 4);
   L->tlist = take(BH * C * kcap * 4);
+  L->order_q = take(BH * C * 4);
+  L->order_kv = take(BH * C * 4);
   L->total = off;
 }
 
@@ -295,6 +299,13 @@ vsa_status run_common(vsa_plan_t P, const void* q, const void* k, const void* v,
   fp.idx = select ? idx_out : idx_in;
   // Top-K rows all hold exactly topk ids: the fine kernel then needs no counts.
   fp.cnt = select ? (P->cfg.topk > 0 ? nullptr : cp.cnt) : cnt_in;
+  // Variable counts: work order longest first per head (schedule.cu).
+  if (fp.cnt) {
+    fp.order = reinterpret_cast<int32_t*>(ws + L.order);
+    if (vsa::launch_schedule(fp.cnt, reinterpret_cast<int32_t*>(ws + L.order), P->BH, P->C, P->kcap, st) !=
+        cudaSuccess)
+      return VSA_ERR_CUDA;
+  }
   fp.oc = cp.oc;
   fp.gate_c = gate_c; fp.gate_f = gate_f;
   fp.out = static_cast<__nv_bfloat16*>(out);
@@ -453,6 +464,13 @@ vsa_status run_backward(vsa_plan_t P, void* bws, size_t bws_bytes, const void* q
   fb.scale_log2 = 1.4426950408889634f / std::sqrt((float)D);
   fb.list = idx; fb.cnt = cnt; fb.off = nullptr;
   fb.cpart0 = cb.dqbar; fb.cpart1 = nullptr;
+  fb.order = nullptr;
+  if (cnt) {
+    fb.order = reinterpret_cast<int32_t*>(bw + BL.order_q);
+    if (vsa::launch_schedule(cnt, reinterpret_cast<int32_t*>(bw + BL.order_q), P->BH, P->C, P->kcap, st) !=
+        cudaSuccess)
+      return VSA_ERR_CUDA;
+  }
   const int grid = fb.n_items < P->num_sms ? fb.n_items : P->num_sms;
   if (!mark(2)) return VSA_ERR_CUDA;
   if (vsa::launch_fine_dq(fb, D, grid, st) != cudaSuccess) return VSA_ERR_CUDA;
@@ -461,6 +479,10 @@ vsa_status run_backward(vsa_plan_t P, void* bws, size_t bws_bytes, const void* q
   if (e != VSA_OK) return e;
   fb.list = tp.tlist; fb.cnt = tp.tcnt; fb.off = tp.toff;
   fb.cpart0 = cb.dkbar; fb.cpart1 = cb.dvbar;
+  fb.order = reinterpret_cast<int32_t*>(bw + BL.order_kv);
+  if (vsa::launch_schedule(tp.tcnt, reinterpret_cast<int32_t*>(bw + BL.order_kv), P->BH, P->C, P->C, st) !=
+      cudaSuccess)
+    return VSA_ERR_CUDA;
   if (!mark(3)) return VSA_ERR_CUDA;
   if (vsa::launch_fine_dkv(fb, D, grid, st) != cudaSuccess) return VSA_ERR_CUDA;
   if (!mark(4)) return VSA_ERR_CUDA;
@@ -935,7 +957,7 @@ vsa_status vsa_stage_times(vsa_plan_t plan, float* ms) {
   return vsa_stage_times_history(plan, ms, 1, &n);
 }
 
-int vsa_kernels_per_run(void) { return 5; }
+int vsa_kernels_per_run(void) { return 5; }  // top-K; variable counts add the schedule kernel
 
 vsa_status vsa_measure_l2_read(const void* buf, size_t bytes, int passes, int* status, void* stream) {
   if (!buf || !status || passes < 1 || bytes < 16384) return VSA_ERR_INVALID_ARG;

@@ -252,13 +252,24 @@ struct Waiter {
   }
 };
 
+// The item at the CTA's position `is`, or -1 past the end. Without an order
+// array the CTA takes items blockIdx.x + is * gridDim.x; with one (variable
+// counts) it takes the positions of a serpentine hand-out of the array,
+// which lists each head's items longest first (schedule.cu).
+__device__ __forceinline__ int item_at(const FineParams& p, int is) {
+  const int G = gridDim.x, c = blockIdx.x;
+  const int pos = is * G + ((p.order && (is & 1)) ? G - 1 - c : c);
+  if (pos >= p.n_items) return -1;
+  return p.order ? p.order[pos] : pos;
+}
+
 // Selected-cube count of an item as stored (validated when the item is reached).
 __device__ __forceinline__ int raw_count(const FineParams& p, int item) {
-  if (item >= p.n_items) return 0;
+  if (item < 0) return 0;
   return p.cnt ? p.cnt[item] : p.kcap;
 }
 
-// Position in the CTA's sequence of steps (items blockIdx.x + is * gridDim.x).
+// Position in the CTA's sequence of steps (items item_at(p, is)).
 // The count of the next item is loaded one item ahead, so no role stalls on
 // it at an item boundary.
 struct Cursor {
@@ -272,7 +283,7 @@ struct Cursor {
   bool bad;    // a count outside [1, kcap] was seen (and clamped)
 };
 __device__ __forceinline__ void cursor_enter(const FineParams& p, Cursor& c, int n_raw) {
-  c.live = c.item < p.n_items;
+  c.live = c.item >= 0;
   int n = n_raw;
   if (c.live && (n < 1 || n > p.kcap)) {
     c.bad = true;
@@ -284,18 +295,18 @@ __device__ __forceinline__ void cursor_enter(const FineParams& p, Cursor& c, int
 }
 __device__ __forceinline__ void cursor_init(const FineParams& p, Cursor& c) {
   c.is = 0;
-  c.item = blockIdx.x;
+  c.item = item_at(p, 0);
   c.bad = false;
   const int n0 = raw_count(p, c.item);
-  c.n_next = raw_count(p, c.item + gridDim.x);
+  c.n_next = raw_count(p, item_at(p, 1));
   cursor_enter(p, c, n0);
 }
 __device__ __forceinline__ void cursor_next(const FineParams& p, Cursor& c) {
   if (++c.t < c.ntiles) return;
   c.is += 1;
-  c.item += gridDim.x;
+  c.item = item_at(p, c.is);
   const int n_raw = c.n_next;
-  c.n_next = raw_count(p, c.item + gridDim.x);
+  c.n_next = raw_count(p, item_at(p, c.is + 1));
   cursor_enter(p, c, n_raw);
 }
 
@@ -620,8 +631,8 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
     int qloads0 = 0, qloads1 = 0;
     // Q of item `is` -> smem buffer is & 1 (TMA, one thread).
     auto load_q = [&](int is) {
-      const int item = blockIdx.x + is * gridDim.x;
-      if (item >= p.n_items) return;
+      const int item = item_at(p, is);
+      if (item < 0) return;
       const int b = is & 1;
       if (b == 0) ++qloads0; else ++qloads1;
       if (est == 0) {
@@ -638,8 +649,8 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
     // row of item `is` -> sh.pre[is & 1]; one cp.async group per call on
     // every thread, so groups stay in the same order everywhere.
     auto prefetch = [&](int is) {
-      const int item = blockIdx.x + is * gridDim.x;
-      if (item < p.n_items && est < 32 + D / 4) {
+      const int item = item_at(p, is);
+      if (item >= 0 && est < 32 + D / 4) {
         const int bh = item / C, ci = item - bh * C;
         Pre& pr = sh.pre[is & 1];
         if (est < 32) {
@@ -658,8 +669,8 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
     load_q(0);
     load_q(1);
     prefetch(0);
-    for (int is = 0; blockIdx.x + is * gridDim.x < p.n_items; ++is) {
-      const int item = blockIdx.x + is * gridDim.x;
+    for (int is = 0; item_at(p, is) >= 0; ++is) {
+      const int item = item_at(p, is);
       const int bh = item / C, ci = item - bh * C;
       const int ct = ci / (Hc * Wc), ch = (ci / Wc) % Hc, cw = ci % Wc;
       const int ob = is & 1;

@@ -93,7 +93,18 @@ struct Waiter {
   __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) const { mbar_wait(bar, parity, limit); }
 };
 
-// One item's position: items blockIdx.x + is * gridDim.x of n_items; n steps.
+// The item at the CTA's position `is`, or -1 past the end: without an order
+// array items blockIdx.x + is * gridDim.x; with one, the positions of a
+// serpentine hand-out of the array (each head's items longest first,
+// schedule.cu).
+__device__ __forceinline__ int item_at(const BwdFineParams& p, int is) {
+  const int G = gridDim.x, c = blockIdx.x;
+  const int pos = is * G + ((p.order && (is & 1)) ? G - 1 - c : c);
+  if (pos >= p.n_items) return -1;
+  return p.order ? p.order[pos] : pos;
+}
+
+// One item's position: the item at position is; n steps.
 struct Cur {
   int is, item, n, t;
   bool live, bad;
@@ -101,7 +112,7 @@ struct Cur {
 
 // dQ kernel: counts from cnt (or kcap), validated to [1, kcap].
 __device__ __forceinline__ void dq_enter(const BwdFineParams& p, Cur& c) {
-  c.live = c.item < p.n_items;
+  c.live = c.item >= 0;
   int n = c.live ? (p.cnt ? p.cnt[c.item] : p.kcap) : 0;
   if (c.live && (n < 1 || n > p.kcap)) {
     c.bad = true;
@@ -112,7 +123,7 @@ __device__ __forceinline__ void dq_enter(const BwdFineParams& p, Cur& c) {
 }
 // dK/dV kernel: counts from the transposed lists, in [0, C].
 __device__ __forceinline__ void dkv_enter(const BwdFineParams& p, Cur& c) {
-  c.live = c.item < p.n_items;
+  c.live = c.item >= 0;
   int n = c.live ? p.cnt[c.item] : 0;
   n = n < 0 ? 0 : (n > p.C ? p.C : n);
   c.n = n;
@@ -121,7 +132,7 @@ __device__ __forceinline__ void dkv_enter(const BwdFineParams& p, Cur& c) {
 template <bool DKV>
 __device__ __forceinline__ void cur_init(const BwdFineParams& p, Cur& c) {
   c.is = 0;
-  c.item = blockIdx.x;
+  c.item = item_at(p, 0);
   c.bad = false;
   if (DKV) dkv_enter(p, c); else dq_enter(p, c);
 }
@@ -129,7 +140,7 @@ __device__ __forceinline__ void cur_init(const BwdFineParams& p, Cur& c) {
 template <bool DKV>
 __device__ __forceinline__ void cur_next_item(const BwdFineParams& p, Cur& c) {
   c.is += 1;
-  c.item += gridDim.x;
+  c.item = item_at(p, c.is);
   if (DKV) dkv_enter(p, c); else dq_enter(p, c);
 }
 
@@ -472,13 +483,13 @@ __global__ void __launch_bounds__(kThreads, 1) fine_dq_kernel(const __grid_const
     uint8_t* stage = tiles + L::OFF_STAGE;
     const int Hc = p.H >> 2, Wc = p.W >> 2;
     auto prefetch = [&](int is) {
-      const int item = blockIdx.x + is * gridDim.x;
-      if (item < p.n_items && est < D / 4) cp_async16(&sh.cpre[is & 1][4 * est], p.cpart0 + (size_t)item * D + 4 * est);
+      const int item = item_at(p, is);
+      if (item >= 0 && est < D / 4) cp_async16(&sh.cpre[is & 1][4 * est], p.cpart0 + (size_t)item * D + 4 * est);
       cp_async_commit();
     };
     prefetch(0);
-    for (int is = 0; blockIdx.x + is * gridDim.x < p.n_items; ++is) {
-      const int item = blockIdx.x + is * gridDim.x;
+    for (int is = 0; item_at(p, is) >= 0; ++is) {
+      const int item = item_at(p, is);
       const int bh = item / C, ci = item - bh * C;
       const int ct = ci / (Hc * Wc), ch = (ci / Wc) % Hc, cw = ci % Wc;
       prefetch(is + 1);
@@ -768,8 +779,8 @@ __global__ void __launch_bounds__(kThreads, 1) fine_dkv_kernel(const __grid_cons
     uint8_t* stage = tiles + L::OFF_STAGE;
     const int Hc = p.H >> 2, Wc = p.W >> 2;
     auto prefetch = [&](int is) {
-      const int item = blockIdx.x + is * gridDim.x;
-      if (item < p.n_items && est < D / 2) {
+      const int item = item_at(p, is);
+      if (item >= 0 && est < D / 2) {
         const int which = est / (D / 4), e = est % (D / 4);
         cp_async16(&sh.cpre[is & 1][which][4 * e], (which ? p.cpart1 : p.cpart0) + (size_t)item * D + 4 * e);
       }

@@ -60,6 +60,7 @@ struct FineParams {
   CUtensorMap tm_out;
   const int32_t* idx;            // [BH, C, kcap]
   const int32_t* cnt;            // [BH, C] or null (then every row has kcap ids)
+  const int32_t* order;          // [BH * C] item order (schedule.cu), or null: items in index order
   const float* oc;               // [BH, C, D]
   const float* gate_c;           // [BH, N]
   const float* gate_f;           // [BH, N]
@@ -139,6 +140,7 @@ struct BwdFineParams {
   const int32_t* list;   // dQ: idx [BH * C, kcap]; dK/dV: the flat transposed lists
   const int32_t* cnt;    // dQ: counts or null (kcap each); dK/dV: tcnt
   const int32_t* off;    // dK/dV: toff; dQ: null
+  const int32_t* order;  // [BH * C] item order (schedule.cu), or null: items in index order
   const float* qstat;    // [BH * C, 2, 64]
   const float* cpart0;   // [BH * C, D] coarse-path gradient rows: dQ kernel dq_bar; dK/dV kernel dk_bar
   const float* cpart1;   // dK/dV kernel dv_bar
@@ -157,6 +159,7 @@ cudaError_t launch_coarse_bwd(const CoarseBwdParams& p, cudaStream_t st);
 cudaError_t launch_tlists(const TlistParams& p, cudaStream_t st);
 cudaError_t launch_fine_dq(const BwdFineParams& p, int D, int grid, cudaStream_t st);
 cudaError_t launch_fine_dkv(const BwdFineParams& p, int D, int grid, cudaStream_t st);
+cudaError_t launch_schedule(const int32_t* len, int32_t* order, int BH, int C, int maxlen, cudaStream_t st);
 cudaError_t launch_l2_read(const void* buf, size_t bytes, int passes, int* status, int grid, cudaStream_t st);
 
 }  // namespace vsa

@@ -40,8 +40,8 @@ class Config(ctypes.Structure):
 
 class WorkspaceLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in ("q_cube", "k_cube", "v_cube", "q_pool", "k_pool", "v_pool",
-                                               "o_coarse", "s_coarse", "pool_split", "p_split", "cnt", "err",
-                                               "total")]
+                                               "o_coarse", "s_coarse", "pool_split", "p_split", "cnt", "order",
+                                               "err", "total")]
 
 
 _lib = None
