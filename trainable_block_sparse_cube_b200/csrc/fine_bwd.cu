@@ -14,6 +14,9 @@
 //   dQ kernel   one item = one query cube; steps over its selected KV cubes.
 //               S = Q K^T and dP = dO V^T (M=64, N=64, SS), dS in TMEM as bf16,
 //               dQ += dS K (M=64, N=D, TS: dS from TMEM, K as an MN-major B).
+//               S and dP buffers are released when read, dS has buffers of
+//               its own, so the S product of a later step never waits for
+//               the dQ product of an earlier one.
 //   dK/dV kernel one item = one KV cube; steps over the query cubes that
 //               selected it (transposed lists). S^T = K Q^T and dP^T = V dO^T
 //               (M=64, N=64, SS), P^T and dS^T in TMEM as bf16,
@@ -24,10 +27,11 @@
 //
 // The eight elementwise warps form two groups that take alternate steps
 // (group g: the steps j with j % 2 == g), so the TMEM round trips of two
-// steps overlap; a warp handles all 64 columns of its lane quarter and writes
-// its 32 packed bf16-pair columns over the first 32 fp32 columns it has
-// already read (no other warp reads that quarter of the buffer). The MMA that
-// reads them takes its K = 16 slices at packed columns 8k.
+// steps overlap; a warp handles all 64 columns of its lane quarter. Its 32
+// packed bf16-pair columns go to a dS buffer of their own (dQ kernel) or over
+// the first 32 fp32 columns it has already read (dK/dV kernel: no other warp
+// reads that quarter of the buffer). The MMA that reads them takes its
+// K = 16 slices at packed columns 8k.
 //
 // Warp roles (512 threads), both kernels:
 //   warp 0      TMA producer (tiles and the per-query statistics)
@@ -237,14 +241,21 @@ struct DqL {
   static constexpr int BYTES = OFF_STAT + 2 * 512;
   static constexpr int SMEM = BYTES + 1024;
 };
-constexpr int kNb = 3;  // S / dP buffers in the dQ kernel
-// TMEM columns (dQ kernel): S buffer b at 64 b, dP buffer b at 192 + 64 b, dQ at 384.
-constexpr uint32_t kQS = 0, kQP = 192, kQAcc = 384;
+// dQ kernel tensor memory: two fp32 S and two fp32 dP buffers (64 columns
+// each; step j uses buffer j % 2, read by the elementwise group j % 2), four
+// bf16 dS buffers (32 columns; step j uses j % 4) and the dQ accumulator.
+// The S and dP buffers are free as soon as the elementwise warps have read
+// them, so S(j + 2) does not wait for the dQ product of step j; only the dS
+// buffers wait for it, four steps later.
+constexpr int kNb = 2;   // S / dP buffers
+constexpr int kNds = 4;  // dS buffers
+constexpr uint32_t kQS = 0, kQP = 128, kQdS = 256, kQAcc = 384;
 
 struct __align__(8) DqBars {
   uint64_t k_full[8], k_empty[8], v_full[8], v_empty[8];  // rings of DqL<D>::KS / VS slots
   uint64_t q_full[2], q_empty[2];
-  uint64_t s_full[kNb], dp_full[kNb], ds_full[kNb], dp_free[kNb], sp_free[kNb];
+  uint64_t s_full[kNb], dp_full[kNb], s_free[kNb], dp_free[kNb];
+  uint64_t ds_full[kNds], ds_free[kNds];
   uint64_t acc_full, acc_empty;
   uint64_t drain[3];
 };
@@ -273,9 +284,12 @@ __global__ void __launch_bounds__(kThreads, 1) fine_dq_kernel(const __grid_const
     for (int b = 0; b < kNb; ++b) {
       mbar_init(&B.s_full[b], 1);
       mbar_init(&B.dp_full[b], 1);
-      mbar_init(&B.ds_full[b], 4);
+      mbar_init(&B.s_free[b], 4);
       mbar_init(&B.dp_free[b], 4);
-      mbar_init(&B.sp_free[b], 1);
+    }
+    for (int d = 0; d < kNds; ++d) {
+      mbar_init(&B.ds_full[d], 4);
+      mbar_init(&B.ds_free[d], 1);
     }
     mbar_init(&B.acc_full, 1);
     mbar_init(&B.acc_empty, 4);
@@ -355,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1) fine_dq_kernel(const __grid_const
       const uint64_t adesc0 = sdesc_sw128(smem_u32(tiles + (is_s ? L::OFF_Q : L::OFF_DO)), 16, 1024);
       const uint64_t bdesc0 = sdesc_sw128(smem_u32(tiles + (is_s ? L::OFF_K : L::OFF_V)), 16, 1024);
       uint64_t* full = is_s ? B.k_full : B.v_full;
-      uint64_t* freed = is_s ? B.sp_free : B.dp_free;
+      uint64_t* freed = is_s ? B.s_free : B.dp_free;
       uint64_t* done = is_s ? B.s_full : B.dp_full;
       bool aborted = false, issued = false;
       int j = 0, b = 0, u = 0;
@@ -399,13 +413,13 @@ __global__ void __launch_bounds__(kThreads, 1) fine_dq_kernel(const __grid_const
       constexpr uint32_t idesc = idesc_bf16_f32(64, D, false, true);
       const uint64_t kdesc0 = sdesc_sw128(smem_u32(tiles + L::OFF_K), 8192, 1024);  // MN-major K
       bool aborted = false, issued = false;
-      int j = 0, b = 0, u = 0;
+      int j = 0, d = 0, ud = 0;  // CTA step, its dS buffer and use count
       Cur c;
       cur_init<false>(p, c);
       while (c.live && !aborted) {
         for (int t = 0; t < c.n; ++t) {
           const int ks = j % L::KS;
-          if ((t == 0 && c.is >= 1 && !W.wait(&B.acc_empty, (c.is - 1) & 1)) || !W.wait(&B.ds_full[b], u & 1)) {
+          if ((t == 0 && c.is >= 1 && !W.wait(&B.acc_empty, (c.is - 1) & 1)) || !W.wait(&B.ds_full[d], ud & 1)) {
             aborted = true;
             break;
           }
@@ -413,14 +427,14 @@ __global__ void __launch_bounds__(kThreads, 1) fine_dq_kernel(const __grid_const
           const uint64_t kd = kdesc0 + (uint64_t)((ks * L::TILE) >> 4);
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            mma_bf16_ts(tmem + kQAcc, tmem + kQS + 64u * b + packed_col(k), kd + (uint64_t)((k * 2048) >> 4), idesc,
+            mma_bf16_ts(tmem + kQAcc, tmem + kQdS + 32u * d + packed_col(k), kd + (uint64_t)((k * 2048) >> 4), idesc,
                         (t > 0 || k > 0) ? 1u : 0u);
-          mma_commit(&B.sp_free[b]);
+          mma_commit(&B.ds_free[d]);
           mma_commit(&B.k_empty[ks]);
           if (t == c.n - 1) mma_commit(&B.acc_full);
           issued = true;
           ++j;
-          if (++b == kNb) { b = 0; ++u; }
+          if (++d == kNds) { d = 0; ++ud; }
         }
         if (aborted) break;
         cur_next_item<false>(p, c);
@@ -433,11 +447,13 @@ __global__ void __launch_bounds__(kThreads, 1) fine_dq_kernel(const __grid_const
     __syncwarp();
   } else if (warp < 12) {
     // ------------------------------------------------------------ P, dS
+    // Group grp takes the steps j with j % 2 == grp, i.e. S / dP buffer grp.
     const int quarter = warp & 3, grp = (warp - 4) >> 2;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const int ra = quarter * 16 + (lane >> 2);
     const float sl2 = p.scale_log2;
-    int j = 0, b = 0, u = 0;  // CTA step, its S/dP buffer and use count
+    const int b = grp;
+    int j = 0;  // CTA step
     Cur c;
     cur_init<false>(p, c);
     while (c.live) {
@@ -447,28 +463,33 @@ __global__ void __launch_bounds__(kThreads, 1) fine_dq_kernel(const __grid_const
       const float l0 = stat[ra], l1 = stat[ra + 8], d0 = stat[64 + ra], d1 = stat[64 + ra + 8];
       __syncwarp();
       if (lane == 0) mbar_arrive(&B.q_empty[qb]);
-      for (int t = 0; t < c.n; ++t) {
-        if ((j & 1) == grp) {
-          W.wait(&B.s_full[b], u & 1);
-          W.wait(&B.dp_full[b], u & 1);
-          tc_fence_after();
-          uint32_t sr[32], g[32];
-          tmem_ld16x256b_x8(tmem + lane_base + kQS + 64u * b, sr);
-          tmem_ld16x256b_x8(tmem + lane_base + kQP + 64u * b, g);
-          tmem_wait_ld();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&B.dp_free[b]);
-          uint32_t pk_p[16], pk_s[16];
-          p_ds<true>(sr, g, sl2, l0, l1, d0, d1, nullptr, nullptr, 0, pk_p, pk_s);
-          tmem_st16x128b_x8(tmem + lane_base + kQS + 64u * b, pk_s);
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&B.ds_full[b]);
+      for (int t = 0; t < c.n; ++t, ++j) {
+        if ((j & 1) != grp) continue;
+        const int u = j >> 1;                  // use of S / dP buffer b
+        const int d = j % kNds, ud = j / kNds;  // dS buffer and its use
+        W.wait(&B.s_full[b], u & 1);
+        W.wait(&B.dp_full[b], u & 1);
+        tc_fence_after();
+        uint32_t sr[32], g[32];
+        tmem_ld16x256b_x8(tmem + lane_base + kQS + 64u * b, sr);
+        tmem_ld16x256b_x8(tmem + lane_base + kQP + 64u * b, g);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&B.s_free[b]);
+          mbar_arrive(&B.dp_free[b]);
         }
-        ++j;
-        if (++b == kNb) { b = 0; ++u; }
+        uint32_t pk_p[16], pk_s[16];
+        p_ds<true>(sr, g, sl2, l0, l1, d0, d1, nullptr, nullptr, 0, pk_p, pk_s);
+        // dS buffer d is free once the dQ product of step j - 4 completed
+        if (ud >= 1) W.wait(&B.ds_free[d], (ud - 1) & 1);
+        tc_fence_after();
+        tmem_st16x128b_x8(tmem + lane_base + kQdS + 32u * d, pk_s);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&B.ds_full[d]);
       }
       cur_next_item<false>(p, c);
     }
@@ -530,14 +551,22 @@ struct DkvL {
   static constexpr int BYTES = OFF_STAGE + TILE;
   static constexpr int SMEM = BYTES + 1024;
 };
-constexpr int kNt = 2;  // S^T / dP^T buffers in the dK/dV kernel
-// TMEM columns (dK/dV kernel): S^T buffer b at 64 b, dP^T buffer b at 128 + 64 b, dK at 256, dV at 256 + D.
-constexpr uint32_t kTS = 0, kTP = 128, kTAcc = 256;
+// dK/dV kernel tensor memory: one fp32 S^T and one fp32 dP^T buffer (64
+// columns each), released as soon as the elementwise warps have read them;
+// two bf16 buffers of P^T and dS^T (64 columns: P^T at +0, dS^T at +32; step
+// j uses j % 2, written by group j % 2), released by the dV / dK products;
+// dK and dV accumulators (D columns each).
+constexpr uint32_t kTS = 0, kTP = 64, kTPD = 128, kTAcc = 256;
 
 struct __align__(8) DkvBars {
   uint64_t kv_full[2], kv_empty[2];
   uint64_t r_full[4], r_empty[4];
-  uint64_t st_full[kNt], dpt_full[kNt], pt_full[kNt], st_free[kNt];
+  // S^T and dP^T of step g complete on st_full[g % 2] / dpt_full[g % 2]: each
+  // elementwise group waits on its own barrier (a parity wait on a barrier
+  // that completes for both groups in turn could not tell its phase from the
+  // previous one). The buffers are freed in step order (one waiter each).
+  uint64_t st_full[2], dpt_full[2], st_free, dpt_free;
+  uint64_t pd_full[2], pd_free[2];
   uint64_t acc_full, acc_empty;
   uint64_t drain[3];
 };
@@ -562,11 +591,15 @@ __global__ void __launch_bounds__(kThreads, 1) fine_dkv_kernel(const __grid_cons
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) { mbar_init(&B.kv_full[i], 1); mbar_init(&B.kv_empty[i], 2); }
     for (int i = 0; i < L::RS; ++i) { mbar_init(&B.r_full[i], 1); mbar_init(&B.r_empty[i], 1); }
-    for (int b = 0; b < kNt; ++b) {
+    for (int b = 0; b < 2; ++b) {
       mbar_init(&B.st_full[b], 1);
       mbar_init(&B.dpt_full[b], 1);
-      mbar_init(&B.pt_full[b], 4);
-      mbar_init(&B.st_free[b], 1);
+    }
+    mbar_init(&B.st_free, 4);
+    mbar_init(&B.dpt_free, 4);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&B.pd_full[b], 4);
+      mbar_init(&B.pd_free[b], 1);
     }
     mbar_init(&B.acc_full, 1);
     mbar_init(&B.acc_empty, 4);
@@ -647,8 +680,9 @@ __global__ void __launch_bounds__(kThreads, 1) fine_dkv_kernel(const __grid_cons
       const uint64_t adesc0 = sdesc_sw128(smem_u32(tiles + L::OFF_KV + (is_s ? 0 : L::TILE)), 16, 1024);
       const uint64_t bdesc0 = sdesc_sw128(smem_u32(tiles + L::OFF_RING + (is_s ? 0 : L::TILE)), 16, 1024);
       uint64_t* done = is_s ? B.st_full : B.dpt_full;
+      uint64_t* freed = is_s ? &B.st_free : &B.dpt_free;
       bool aborted = false, issued = false;
-      int g = 0, kvu = 0, b = 0, u = 0;
+      int g = 0, kvu = 0;  // CTA step, items with steps
       Cur c;
       cur_init<true>(p, c);
       while (c.live && !aborted) {
@@ -656,8 +690,9 @@ __global__ void __launch_bounds__(kThreads, 1) fine_dkv_kernel(const __grid_cons
           const int kb = kvu & 1;
           for (int t = 0; t < c.n; ++t) {
             const int rs = g % L::RS;
+            // the single fp32 buffer is free once step g - 1 was read
             if ((t == 0 && !W.wait(&B.kv_full[kb], (kvu >> 1) & 1)) ||
-                (u >= 1 && !W.wait(&B.st_free[b], (u - 1) & 1)) || !W.wait(&B.r_full[rs], (g / L::RS) & 1)) {
+                (g >= 1 && !W.wait(freed, (g - 1) & 1)) || !W.wait(&B.r_full[rs], (g / L::RS) & 1)) {
               aborted = true;
               break;
             }
@@ -666,12 +701,11 @@ __global__ void __launch_bounds__(kThreads, 1) fine_dkv_kernel(const __grid_cons
             const uint64_t bd = bdesc0 + (uint64_t)((rs * L::SLOT) >> 4);
 #pragma unroll
             for (int k = 0; k < D / 16; ++k)
-              mma_bf16_ss(tmem + col0 + 64u * b, ad + kmajor_off(k), bd + kmajor_off(k), idesc, k > 0 ? 1u : 0u);
-            mma_commit(&done[b]);
+              mma_bf16_ss(tmem + col0, ad + kmajor_off(k), bd + kmajor_off(k), idesc, k > 0 ? 1u : 0u);
+            mma_commit(&done[g & 1]);
             if (t == c.n - 1) mma_commit(&B.kv_empty[kb]);
             issued = true;
             ++g;
-            if (++b == kNt) { b = 0; ++u; }
           }
           if (aborted) break;
           ++kvu;
@@ -692,33 +726,33 @@ __global__ void __launch_bounds__(kThreads, 1) fine_dkv_kernel(const __grid_cons
       const uint64_t qdesc0 = sdesc_sw128(smem_u32(tiles + L::OFF_RING), 8192, 1024);            // MN-major Q
       const uint64_t ddesc0 = sdesc_sw128(smem_u32(tiles + L::OFF_RING + L::TILE), 8192, 1024);  // MN-major dO
       bool aborted = false, issued = false;
-      int g = 0, acc = 0, b = 0, u = 0;
+      int g = 0, acc = 0;  // CTA step, items with steps
       Cur c;
       cur_init<true>(p, c);
       while (c.live && !aborted) {
         if (c.n > 0) {
           for (int t = 0; t < c.n; ++t) {
-            const int rs = g % L::RS;
-            if ((t == 0 && acc >= 1 && !W.wait(&B.acc_empty, (acc - 1) & 1)) || !W.wait(&B.pt_full[b], u & 1)) {
+            const int rs = g % L::RS, b = g & 1;
+            if ((t == 0 && acc >= 1 && !W.wait(&B.acc_empty, (acc - 1) & 1)) || !W.wait(&B.pd_full[b], (g >> 1) & 1)) {
               aborted = true;
               break;
             }
             tc_fence_after();
             const uint64_t so = (uint64_t)((rs * L::SLOT) >> 4);
+            const uint32_t pd = tmem + kTPD + 64u * b;
 #pragma unroll
             for (int k = 0; k < 4; ++k)  // dV += P^T dO
-              mma_bf16_ts(tmem + kTAcc + D, tmem + kTS + 64u * b + packed_col(k), ddesc0 + so + (uint64_t)((k * 2048) >> 4),
-                          idesc, (t > 0 || k > 0) ? 1u : 0u);
+              mma_bf16_ts(tmem + kTAcc + D, pd + packed_col(k), ddesc0 + so + (uint64_t)((k * 2048) >> 4), idesc,
+                          (t > 0 || k > 0) ? 1u : 0u);
 #pragma unroll
             for (int k = 0; k < 4; ++k)  // dK += dS^T Q
-              mma_bf16_ts(tmem + kTAcc, tmem + kTP + 64u * b + packed_col(k), qdesc0 + so + (uint64_t)((k * 2048) >> 4),
-                          idesc, (t > 0 || k > 0) ? 1u : 0u);
-            mma_commit(&B.st_free[b]);
+              mma_bf16_ts(tmem + kTAcc, pd + 32u + packed_col(k), qdesc0 + so + (uint64_t)((k * 2048) >> 4), idesc,
+                          (t > 0 || k > 0) ? 1u : 0u);
+            mma_commit(&B.pd_free[b]);
             mma_commit(&B.r_empty[rs]);
             if (t == c.n - 1) mma_commit(&B.acc_full);
             issued = true;
             ++g;
-            if (++b == kNt) { b = 0; ++u; }
           }
           if (aborted) break;
           ++acc;
@@ -733,38 +767,44 @@ __global__ void __launch_bounds__(kThreads, 1) fine_dkv_kernel(const __grid_cons
     __syncwarp();
   } else if (warp < 12) {
     // ------------------------------------------------------------ P^T, dS^T
-    // Two S^T / dP^T buffers and two groups: group g always works on buffer g.
+    // Group grp takes the steps g with g % 2 == grp (bf16 buffer grp).
     const int quarter = warp & 3, grp = (warp - 4) >> 2;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const int c0 = 2 * (lane & 3);  // first query column of the thread (plus 8 j)
     const float sl2 = p.scale_log2;
-    int g = 0, b = 0, u = 0;
+    int g = 0;
     Cur c;
     cur_init<true>(p, c);
     while (c.live) {
-      for (int t = 0; t < c.n; ++t) {
-        if (b == grp) {
-          const int rs = g % L::RS;
-          W.wait(&B.r_full[rs], (g / L::RS) & 1);
-          W.wait(&B.st_full[b], u & 1);
-          W.wait(&B.dpt_full[b], u & 1);
-          tc_fence_after();
-          const float* stat = reinterpret_cast<const float*>(tiles + L::OFF_RING + rs * L::SLOT + 2 * L::TILE);
-          uint32_t s[32], gg[32];
-          tmem_ld16x256b_x8(tmem + lane_base + kTS + 64u * b, s);
-          tmem_ld16x256b_x8(tmem + lane_base + kTP + 64u * b, gg);
-          tmem_wait_ld();
-          uint32_t pk_p[16], pk_s[16];
-          p_ds<false>(s, gg, sl2, 0.f, 0.f, 0.f, 0.f, stat, stat + 64, c0, pk_p, pk_s);
-          tmem_st16x128b_x8(tmem + lane_base + kTS + 64u * b, pk_p);
-          tmem_st16x128b_x8(tmem + lane_base + kTP + 64u * b, pk_s);
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&B.pt_full[b]);
+      for (int t = 0; t < c.n; ++t, ++g) {
+        if ((g & 1) != grp) continue;
+        const int rs = g % L::RS;
+        W.wait(&B.r_full[rs], (g / L::RS) & 1);
+        W.wait(&B.st_full[grp], (g >> 1) & 1);
+        W.wait(&B.dpt_full[grp], (g >> 1) & 1);
+        tc_fence_after();
+        const float* stat = reinterpret_cast<const float*>(tiles + L::OFF_RING + rs * L::SLOT + 2 * L::TILE);
+        uint32_t s[32], gg[32];
+        tmem_ld16x256b_x8(tmem + lane_base + kTS, s);
+        tmem_ld16x256b_x8(tmem + lane_base + kTP, gg);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&B.st_free);
+          mbar_arrive(&B.dpt_free);
         }
-        ++g;
-        if (++b == kNt) { b = 0; ++u; }
+        uint32_t pk_p[16], pk_s[16];
+        p_ds<false>(s, gg, sl2, 0.f, 0.f, 0.f, 0.f, stat, stat + 64, c0, pk_p, pk_s);
+        // bf16 buffer grp is free once the dV / dK products of step g - 2 completed
+        if (g >= 2) W.wait(&B.pd_free[grp], ((g >> 1) - 1) & 1);
+        tc_fence_after();
+        tmem_st16x128b_x8(tmem + lane_base + kTPD + 64u * grp, pk_p);
+        tmem_st16x128b_x8(tmem + lane_base + kTPD + 64u * grp + 32u, pk_s);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&B.pd_full[grp]);
       }
       cur_next_item<true>(p, c);
     }
