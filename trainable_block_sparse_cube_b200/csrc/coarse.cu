@@ -126,6 +126,65 @@ __device__ __forceinline__ void row_softmax(const CoarseParams& p, int row, uint
   }
 }
 
+// row_softmax for C <= 1024 with the row in registers: lane t holds columns
+// 64u + 2t and 64u + 2t + 1 (u < C/64 rounded up), so every score is read
+// once, every exponential computed once, and the probabilities' three terms
+// are stored as bf16 pairs. The keys still go to shared memory for the
+// selection.
+__device__ __forceinline__ void row_softmax_regs(const CoarseParams& p, int row, uint32_t* keys, int lane, float& mb,
+                                                 float& l, uint32_t& lkmax) {
+  const int C = p.C;
+  const float* srow = p.s + (size_t)row * C;
+  float v[32];
+  float lm = -INFINITY;
+  lkmax = 0;
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    const int j = 64 * u + 2 * lane;
+    v[2 * u] = j < C ? srow[j] : -INFINITY;
+    v[2 * u + 1] = j + 1 < C ? srow[j + 1] : -INFINITY;
+  }
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    const int j = 64 * u + 2 * lane;
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      if (j + h < C) {
+        const uint32_t k = order_key(v[2 * u + h]);
+        keys[j + h] = k;
+        lkmax = max(lkmax, k);
+        lm = fmaxf(lm, v[2 * u + h]);
+      }
+  }
+  mb = warp_max(lm) * kLog2e;
+  float ls = 0.f;
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    v[e] = fast_exp2(fmaf(v[e], kLog2e, -mb));  // -inf (padding) -> 0
+    ls += v[e];
+  }
+  l = warp_sum(ls);
+  const float inv_l = 1.0f / l;
+  const size_t plane = (size_t)p.BH * C * p.Cp;
+  __nv_bfloat16* prow = p.psplit + (size_t)row * p.Cp;
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    const int j = 64 * u + 2 * lane;
+    if (j < p.Cp) {  // Cp is a multiple of 8: the pair j, j + 1 lies inside the row
+      float x0 = v[2 * u] * inv_l, x1 = v[2 * u + 1] * inv_l;
+#pragma unroll
+      for (int t = 0; t < 3; ++t) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+        const float2 back = __bfloat1622float2(h);
+        x0 -= back.x;
+        x1 -= back.y;
+        *reinterpret_cast<__nv_bfloat162*>(prow + t * plane + j) = h;
+      }
+    }
+  }
+  __syncwarp();
+}
+
 // Top-K emission for Kt <= 32 from the candidates (keys at or above the lower
 // bound lo, with their ids, in ascending id order, NS slots per lane): the
 // Kt-th largest key T by the MSB-first search below the bits that lo and the
@@ -184,7 +243,8 @@ __device__ __forceinline__ void topk_from_candidates(const uint32_t* ckey, const
 // maxima bounds the K-th largest key from below, and the search runs over the
 // candidates at or above it, compacted in place; larger K, or more than
 // kCandCap candidates, take the bit search over all keys.
-__global__ void __launch_bounds__(256, 4) coarse_select_topk_kernel(const CoarseParams p) {
+template <bool REGS>
+__global__ void __launch_bounds__(256, REGS ? 2 : 4) coarse_select_topk_kernel(const CoarseParams p) {
   extern __shared__ __align__(16) uint8_t dyn[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * 8 + warp;
@@ -196,7 +256,8 @@ __global__ void __launch_bounds__(256, 4) coarse_select_topk_kernel(const Coarse
   const uint32_t lt_mask = (1u << lane) - 1u;
   float mb, l;
   uint32_t lkmax;
-  row_softmax(p, row, keys, lane, mb, l, lkmax);
+  if (REGS) row_softmax_regs(p, row, keys, lane, mb, l, lkmax);
+  else row_softmax(p, row, keys, lane, mb, l, lkmax);
   if (!p.do_select) return;
   int32_t* irow = p.idx + (size_t)row * p.kcap;
   // Lower bound lo of the Kt-th largest key (for Kt <= 32: every lane with a
@@ -366,10 +427,18 @@ __global__ void __launch_bounds__(256, 2) coarse_select_topp_kernel(const Coarse
 // Every wait is bounded; a wait that gives up records kErrTimeout.
 template <int KIND, int D>
 struct TcShape {
+  // Bf16 terms used per operand and products summed: the scores decide
+  // integer selections and keep all three terms (six products, dropped terms
+  // below 2^-24 relative). The coarse output decides nothing and is checked
+  // against the fp64 oracle at 1e-4: hi + mid (16 significant bits, error
+  // <= 2^-18 relative) and the products hi.hi, hi.mid, mid.hi leave an error
+  // of a few 2^-18 relative, about 2e-5 absolute for these means.
+  static constexpr int TERMS = KIND == 0 ? 3 : 2;
+  static constexpr int PRODUCTS = KIND == 0 ? 6 : 3;
   static constexpr int NT = KIND == 0 ? 128 : D;    // accumulator columns
   static constexpr int A_BYTES = 128 * 64 * 2;      // one term, 128 rows x 64 K
   static constexpr int B_BYTES = NT * 64 * 2;       // one term
-  static constexpr int STAGE = 3 * (A_BYTES + B_BYTES);
+  static constexpr int STAGE = TERMS * (A_BYTES + B_BYTES);
   // Scores: K = D is one or two 64-column chunks, so a single stage lets two
   // CTAs share an SM and overlap each other's loads, MMAs and epilogue.
   // Output: K = Cp is up to 64 chunks, double-buffered.
@@ -408,7 +477,7 @@ __global__ void __launch_bounds__(128, KIND == 0 ? 2 : 1) coarse_tc_kernel(const
   tc_fence_after();
   const uint32_t tmem = tmem_base;
   auto a_tile = [&](int st, int t) { return tiles + st * S::STAGE + t * S::A_BYTES; };
-  auto b_tile = [&](int st, int t) { return tiles + st * S::STAGE + 3 * S::A_BYTES + t * S::B_BYTES; };
+  auto b_tile = [&](int st, int t) { return tiles + st * S::STAGE + S::TERMS * S::A_BYTES + t * S::B_BYTES; };
 
   if (warp == 0 && lane == 0) {
     const CUtensorMap* ta = KIND == 0 ? &p.tm_qs : &p.tm_ps;
@@ -422,7 +491,7 @@ __global__ void __launch_bounds__(128, KIND == 0 ? 2 : 1) coarse_tc_kernel(const
       }
       mbar_arrive_expect_tx(&full[st], S::STAGE);
       ++armed;
-      for (int t = 0; t < 3; ++t) {
+      for (int t = 0; t < S::TERMS; ++t) {
         tma_load_3d(a_tile(st, t), ta, &full[st], 64 * c, m0, t * BH + bh);
         if (KIND == 0) {
           tma_load_3d(b_tile(st, t), tb, &full[st], 64 * c, n0, t * BH + bh);
@@ -437,7 +506,10 @@ __global__ void __launch_bounds__(128, KIND == 0 ? 2 : 1) coarse_tc_kernel(const
   } else if (warp == 1 && lane == 0) {
     constexpr uint32_t idesc = idesc_bf16_f32(128, S::NT, false, KIND == 1);
     // Term pairs (A term, B term) of the six products kept.
-    constexpr int pa[6] = {2, 0, 1, 1, 0, 0}, pb[6] = {0, 2, 1, 0, 1, 0};
+    // term pairs, smallest products first: all six pairs above 2^-24 (scores),
+    // or mid.hi, hi.mid, hi.hi (output)
+    constexpr int pa[6] = {KIND == 0 ? 2 : 1, 0, 1, 1, 0, 0}, pb[6] = {0, KIND == 0 ? 2 : 1, 1, 0, 1, 0};
+    constexpr int q0 = 6 - S::PRODUCTS;
     bool ok = true;
     for (int c = 0; c < nch && ok; ++c) {
       const int st = c % S::NS;
@@ -450,12 +522,12 @@ __global__ void __launch_bounds__(128, KIND == 0 ? 2 : 1) coarse_tc_kernel(const
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
-        for (int q = 0; q < 6; ++q) {
+        for (int q = q0; q < 6; ++q) {
           const uint64_t ad = sdesc_sw128(smem_u32(a_tile(st, pa[q])), 16, 1024) + (uint64_t)((kk * 32) >> 4);
           uint64_t bd;
           if (KIND == 0) bd = sdesc_sw128(smem_u32(b_tile(st, pb[q])), 16, 1024) + (uint64_t)((kk * 32) >> 4);
           else bd = sdesc_sw128(smem_u32(b_tile(st, pb[q])), 8192, 1024) + (uint64_t)((kk * 2048) >> 4);
-          mma_bf16_ss(tmem, ad, bd, idesc, (c > 0 || kk > 0 || q > 0) ? 1u : 0u);
+          mma_bf16_ss(tmem, ad, bd, idesc, (c > 0 || kk > 0 || q > q0) ? 1u : 0u);
         }
       mma_commit(&empty[st]);
     }
@@ -520,11 +592,16 @@ cudaError_t launch_select_topk(const CoarseParams& p, cudaStream_t st) {
   const int rows = p.BH * p.C;
   const size_t smem = (size_t)8 * ((p.C + 31) / 32 * 32 + kCandCap) * 4;
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(coarse_select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    cudaError_t e = p.C <= 1024 ? cudaFuncSetAttribute(coarse_select_topk_kernel<true>,
+                                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
+                                : cudaFuncSetAttribute(coarse_select_topk_kernel<false>,
+                                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  coarse_select_topk_kernel<<<(rows + 7) / 8, 256, smem, st>>>(p);
+  if (p.C <= 1024)
+    coarse_select_topk_kernel<true><<<(rows + 7) / 8, 256, smem, st>>>(p);
+  else
+    coarse_select_topk_kernel<false><<<(rows + 7) / 8, 256, smem, st>>>(p);
   return cudaGetLastError();
 }
 
