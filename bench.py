@@ -43,7 +43,7 @@ from trainable_block_sparse_cube_b200 import replicas, synth  # noqa: E402
 
 METRIC = "VSA fwd ms/call & sparse TFLOP/s (% bf16 TC peak) at 61,440 tokens, K=32"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
-FINE_SOURCES = ["fine.cu", "sm100_ptx.cuh", "poly_exp2.cuh"]   # the fine kernel's own code
+FINE_SOURCES = ["fine.cu", "sm100_ptx.cuh"]   # the fine kernel's own code
 PROFILE_JSON = os.path.join(ROOT, "profiles", "fine_attention_long61k_k32.json")
 SWEEP = ["tiny", "pretrain16k", "long61k_k16", "long61k_k32", "dynamic61k", "large77k"]
 FINE_FLOP_PER_L2_BYTE = 64.0   # 4*64*64*D FLOP per 64-token K+V tile pair of 2*64*D*2 bytes

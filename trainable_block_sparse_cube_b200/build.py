@@ -28,7 +28,7 @@ def _nvcc() -> str:
 
 def build(verbose: bool = False, force: bool = False) -> str:
     srcs = [os.path.join(HERE, "csrc", s) for s in SRC]
-    deps = srcs + [os.path.join(HERE, "csrc", h) for h in ("vsa_common.cuh", "sm100_ptx.cuh", "poly_exp2.cuh")]
+    deps = srcs + [os.path.join(HERE, "csrc", h) for h in ("vsa_common.cuh", "sm100_ptx.cuh")]
     deps.append(os.path.join(os.path.dirname(HERE), "include", "vsa.h"))
     if not force and os.path.exists(LIB):
         t = os.path.getmtime(LIB)
