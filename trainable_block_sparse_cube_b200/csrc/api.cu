@@ -261,7 +261,7 @@ vsa_status run_common(vsa_plan_t P, const void* q, const void* k, const void* v,
   gp.BH = P->BH; gp.C = P->C; gp.H = c.H; gp.W = c.W; gp.N = P->N;
   cudaEvent_t* ev = P->timing ? P->ev + 4 * (P->timed_runs % P->ring) : nullptr;
   if (ev && cudaEventRecord(ev[0], st) != cudaSuccess) return VSA_ERR_CUDA;
-  if (vsa::launch_gather(gp, c.D, st) != cudaSuccess) return VSA_ERR_CUDA;
+  if (vsa::launch_gather(gp, c.D, P->num_sms, st) != cudaSuccess) return VSA_ERR_CUDA;
   if (ev && cudaEventRecord(ev[1], st) != cudaSuccess) return VSA_ERR_CUDA;
 
   vsa::CoarseParams cp{};
@@ -378,7 +378,7 @@ vsa_status run_backward(vsa_plan_t P, void* bws, size_t bws_bytes, const void* q
   for (int t = 0; t < 3; ++t)
     gp.split[t] = reinterpret_cast<__nv_bfloat16*>(ws + L.pool_split + (size_t)t * 3 * P->BH * P->C * D * 2);
   gp.BH = P->BH; gp.C = P->C; gp.H = c.H; gp.W = c.W; gp.N = P->N;
-  if (vsa::launch_gather(gp, D, st) != cudaSuccess) return VSA_ERR_CUDA;
+  if (vsa::launch_gather(gp, D, P->num_sms, st) != cudaSuccess) return VSA_ERR_CUDA;
   vsa::CoarseParams cp{};
   cp.tm_qs = P->tm_qs; cp.tm_ks = P->tm_ks; cp.tm_vs = P->tm_vs; cp.tm_ps = P->tm_ps;
   cp.psplit = reinterpret_cast<__nv_bfloat16*>(ws + L.p_split);

@@ -9,27 +9,28 @@
 // kernel reads q straight from its raster layout, so q's copy is written
 // only when a plan asks for it for inspection.
 //
-// One warp per (tensor, head, cube). A raster row of D bf16 is D*2 bytes; a
-// lane moves 16 bytes, so D/8 lanes cover a row and a warp covers 32/(D/8)
-// rows per step. Four consecutive w positions of a cube are contiguous in the
+// One warp per (tensor, head, cube) unit at a time: the grid is sized to
+// about eight 256-thread blocks per SM and each warp strides over the units
+// (tensor fastest, so the q, k and v of a cube go to neighbouring warps),
+// which avoids the partial last wave of a one-unit-per-warp grid. A raster
+// row of D bf16 is D*2 bytes; a lane moves 16 bytes, so D/8 lanes cover a row
+// and a warp covers 32/(D/8) rows per step. Four consecutive w positions of a cube are contiguous in the
 // raster layout (4*D*2 bytes), and every read and write is a full 16-byte
 // vector. The pool sums are kept per lane in fp32 and combined with shuffles.
 #include "vsa_common.cuh"
 
 namespace vsa {
 
+// One (tensor, head, cube) unit: the cube's 64 raster rows of tensor
+// `tensor` -> its fp32 mean and three bf16 terms, and the cube-major copy
+// when the tensor has one.
 template <int D>
-__global__ void __launch_bounds__(256) gather_pool_kernel(const GatherParams p) {
+__device__ __forceinline__ void gather_pool_unit(const GatherParams& p, int tensor, int bh, int c, int sub, int chunk) {
   constexpr int LPR = D / 8;        // lanes per row
   constexpr int RPS = 32 / LPR;     // rows per warp step
   constexpr int STEPS = kCube / RPS;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int c = blockIdx.x * 8 + warp;
-  const int bh = blockIdx.y, tensor = blockIdx.z;
-  if (c >= p.C) return;
-  const int sub = lane / LPR, chunk = lane % LPR;
   const __nv_bfloat16* src = p.src[tensor] + (size_t)bh * p.N * D + chunk * 8;
-  const bool copy = p.dst[tensor] != nullptr;  // uniform over the grid's z slice
+  const bool copy = p.dst[tensor] != nullptr;
   __nv_bfloat16* dst = copy ? p.dst[tensor] + ((size_t)bh * p.C + c) * kCube * D + chunk * 8 : nullptr;
 
   float acc[8];
@@ -94,8 +95,24 @@ __global__ void __launch_bounds__(256) gather_pool_kernel(const GatherParams p) 
   }
 }
 
-cudaError_t launch_gather(const GatherParams& p, int D, cudaStream_t st) {
-  dim3 grid((p.C + 7) / 8, p.BH, 3);
+template <int D>
+__global__ void __launch_bounds__(256) gather_pool_kernel(const GatherParams p) {
+  constexpr int LPR = D / 8;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sub = lane / LPR, chunk = lane % LPR;
+  const int units = 3 * p.BH * p.C;
+  for (int unit = blockIdx.x * 8 + warp; unit < units; unit += gridDim.x * 8) {
+    const int tensor = unit % 3, rest = unit / 3;
+    const int bh = rest / p.C, c = rest - bh * p.C;
+    gather_pool_unit<D>(p, tensor, bh, c, sub, chunk);
+  }
+}
+
+cudaError_t launch_gather(const GatherParams& p, int D, int num_sms, cudaStream_t st) {
+  const long long units = 3LL * p.BH * p.C;
+  long long blocks = (units + 7) / 8;
+  if (blocks > 8LL * num_sms) blocks = 8LL * num_sms;
+  const dim3 grid((unsigned)blocks);
   if (D == 128)
     gather_pool_kernel<128><<<grid, 256, 0, st>>>(p);
   else

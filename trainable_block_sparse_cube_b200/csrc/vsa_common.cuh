@@ -151,7 +151,7 @@ struct BwdFineParams {
   float scale;           // 1 / sqrt(D)
 };
 
-cudaError_t launch_gather(const GatherParams& p, int D, cudaStream_t st);
+cudaError_t launch_gather(const GatherParams& p, int D, int num_sms, cudaStream_t st);
 cudaError_t launch_coarse(const CoarseParams& p, cudaStream_t st);
 cudaError_t launch_fine(const FineParams& p, int D, int grid, cudaStream_t st);
 cudaError_t launch_bwd_prep(const PrepParams& p, int D, cudaStream_t st);
