@@ -267,6 +267,7 @@ vsa_status run_common(vsa_plan_t P, const void* q, const void* k, const void* v,
   vsa::CoarseParams cp{};
   cp.tm_qs = P->tm_qs; cp.tm_ks = P->tm_ks; cp.tm_vs = P->tm_vs; cp.tm_ps = P->tm_ps;
   cp.psplit = reinterpret_cast<__nv_bfloat16*>(ws + L.p_split);
+  cp.p_terms = 2;  // the output product reads hi and mid
   cp.Cp = (int)coarse_pitch(P->C);
   cp.err = reinterpret_cast<int*>(ws + L.err);
   cp.wait_ns = P->wait_ns;
@@ -382,6 +383,7 @@ vsa_status run_backward(vsa_plan_t P, void* bws, size_t bws_bytes, const void* q
   vsa::CoarseParams cp{};
   cp.tm_qs = P->tm_qs; cp.tm_ks = P->tm_ks; cp.tm_vs = P->tm_vs; cp.tm_ps = P->tm_ps;
   cp.psplit = reinterpret_cast<__nv_bfloat16*>(ws + L.p_split);
+  cp.p_terms = 3;  // the coarse backward's products read all three terms
   cp.Cp = (int)coarse_pitch(P->C);
   cp.err = reinterpret_cast<int*>(ws + L.err);
   cp.wait_ns = P->wait_ns;

@@ -17,8 +17,9 @@
 //   1. scores   s = qbar kbar^T / sqrt(D)       [BH, C, C]   (tcgen05, 128 x 128 tiles)
 //   2. select   one warp per row, the row's scores as order-preserving
 //               uint32 keys in shared memory: row max and sum, the
-//               probabilities P written as three bf16 terms, then the
-//               selection. Top-K <= 32: the minimum of the lanes' maxima
+//               probabilities P written as bf16 terms (hi and mid for the
+//               forward's output product, also lo when the backward's
+//               products need them), then the selection. Top-K <= 32: the minimum of the lanes' maxima
 //               bounds the K-th largest key from below, the keys at or above
 //               it are compacted in place (ascending id) and an MSB-first
 //               count search over them finds the K-th largest; larger K, or
@@ -122,7 +123,7 @@ __device__ __forceinline__ void row_softmax(const CoarseParams& p, int row, uint
     const __nv_bfloat16 md = __float2bfloat16_rn(r1);
     prow[j] = h;
     prow[plane + j] = md;
-    prow[2 * plane + j] = __float2bfloat16_rn(r1 - __bfloat162float(md));
+    if (p.p_terms > 2) prow[2 * plane + j] = __float2bfloat16_rn(r1 - __bfloat162float(md));
   }
 }
 
@@ -167,6 +168,7 @@ __device__ __forceinline__ void row_softmax_regs(const CoarseParams& p, int row,
   const float inv_l = 1.0f / l;
   const size_t plane = (size_t)p.BH * C * p.Cp;
   __nv_bfloat16* prow = p.psplit + (size_t)row * p.Cp;
+  const int terms = p.p_terms;
 #pragma unroll
   for (int u = 0; u < 16; ++u) {
     const int j = 64 * u + 2 * lane;
@@ -178,7 +180,7 @@ __device__ __forceinline__ void row_softmax_regs(const CoarseParams& p, int row,
         const float2 back = __bfloat1622float2(h);
         x0 -= back.x;
         x1 -= back.y;
-        *reinterpret_cast<__nv_bfloat162*>(prow + t * plane + j) = h;
+        if (t < terms) *reinterpret_cast<__nv_bfloat162*>(prow + t * plane + j) = h;
       }
     }
   }
@@ -244,7 +246,7 @@ __device__ __forceinline__ void topk_from_candidates(const uint32_t* ckey, const
 // candidates at or above it, compacted in place; larger K, or more than
 // kCandCap candidates, take the bit search over all keys.
 template <bool REGS>
-__global__ void __launch_bounds__(256, REGS ? 2 : 4) coarse_select_topk_kernel(const CoarseParams p) {
+__global__ void __launch_bounds__(256, 4) coarse_select_topk_kernel(const CoarseParams p) {
   extern __shared__ __align__(16) uint8_t dyn[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * 8 + warp;

@@ -36,7 +36,8 @@ struct CoarseParams {
   //   tm_ps: [3 * BH][C][Cp], boxes of 128 rows x 64 columns.
   CUtensorMap tm_qs, tm_ks, tm_vs, tm_ps;
   float* s;            // [BH, C, C] scores
-  __nv_bfloat16* psplit;  // [3, BH, C, Cp] coarse probabilities as three bf16 terms
+  __nv_bfloat16* psplit;  // [3, BH, C, Cp] coarse probabilities as bf16 terms (hi, mid, lo)
+  int p_terms;         // terms of P written: 2 (the forward's output product), 3 (the backward's products)
   float* oc;           // [BH, C, D]
   float* oc_copy;      // optional second destination of oc (may be null)
   int Cp;              // C rounded up to a multiple of 8 (row pitch of psplit)
