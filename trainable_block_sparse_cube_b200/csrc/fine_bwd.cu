@@ -11,12 +11,12 @@
 // summed, for K and V, over every query cube that selected the KV cube.
 //
 // Two kernels, no atomics (deterministic):
-//   dQ kernel   one item = one query cube; steps over its selected KV cubes.
-//               S = Q K^T and dP = dO V^T (M=64, N=64, SS), dS in TMEM as bf16,
-//               dQ += dS K (M=64, N=D, TS: dS from TMEM, K as an MN-major B).
-//               S and dP buffers are released when read, dS has buffers of
-//               its own, so the S product of a later step never waits for
-//               the dQ product of an earlier one.
+//   dQ kernel   one item = one query cube; steps of two of its selected KV
+//               cubes (128 keys). S = Q K^T and dP = dO V^T (M=64, N=128,
+//               SS), dS in TMEM as bf16, dQ += dS K (M=64, N=D, TS: dS from
+//               TMEM, K as an MN-major B). The S and dP buffers are released
+//               when read, dS has buffers of its own, so the S product of the
+//               next step never waits for the dQ product of this one.
 //   dK/dV kernel one item = one KV cube; steps over the query cubes that
 //               selected it (transposed lists). S^T = K Q^T and dP^T = V dO^T
 //               (M=64, N=64, SS), P^T and dS^T in TMEM as bf16,
@@ -25,13 +25,15 @@
 // accumulators use the M=64 TMEM layout (16 lanes of each 32-lane quarter);
 // the softmax-side warps read and write them with the 16-lane shapes.
 //
-// The eight elementwise warps form two groups that take alternate steps
-// (group g: the steps j with j % 2 == g), so the TMEM round trips of two
-// steps overlap; a warp handles all 64 columns of its lane quarter. Its 32
-// packed bf16-pair columns go to a dS buffer of their own (dQ kernel) or over
-// the first 32 fp32 columns it has already read (dK/dV kernel: no other warp
-// reads that quarter of the buffer). The MMA that reads them takes its
-// K = 16 slices at packed columns 8k.
+// Elementwise warps. dQ kernel: all eight work on every step, warp w on the
+// rows of lane quarter w % 4 and key half (w - 4) / 4; their packed bf16-pair
+// columns (32 per warp) go to a dS buffer of their own. dK/dV kernel: two
+// groups of four take alternate steps (group g: the steps j with j % 2 == g),
+// so the TMEM round trips of two steps overlap; a warp handles all 64 columns
+// of its lane quarter and writes its 32 packed columns over the first 32 fp32
+// columns it has already read (no other warp reads that quarter of the
+// buffer). The MMA that reads them takes its K = 16 slices at packed columns
+// 8k.
 //
 // Warp roles (512 threads), both kernels:
 //   warp 0      TMA producer (tiles and the per-query statistics)
@@ -227,38 +229,44 @@ __device__ __forceinline__ void p_ds(const uint32_t (&s)[32], const uint32_t (&g
 }
 
 // ============================================================ dQ kernel
+// Steps of two selected KV cubes (128 keys), as in the forward kernel: per
+// step 8 S MMAs (M=64, N=128), 8 dP MMAs (M=64, N=128) and 8 dQ MMAs (M=64,
+// N=D, K=16 keys each). An odd count loads the last cube twice; the
+// elementwise warps zero the repeated half's dS.
 template <int D>
 struct DqL {
   static constexpr int NH = D / 64;
-  static constexpr int TILE = 64 * D * 2;
-  static constexpr int KS = 4, VS = 3;
+  static constexpr int TILE = 64 * D * 2;               // one cube
+  static constexpr int PAIR = 2 * TILE;                 // one step's K or V (two cubes)
+  static constexpr int KS = 2, VS = 2;
   static constexpr int OFF_Q = 0;                       // Q[2]
   static constexpr int OFF_DO = OFF_Q + 2 * TILE;       // dO[2]
-  static constexpr int OFF_K = OFF_DO + 2 * TILE;       // K ring
-  static constexpr int OFF_V = OFF_K + KS * TILE;       // V ring
-  static constexpr int OFF_STAGE = OFF_V + VS * TILE;   // output staging
+  static constexpr int OFF_K = OFF_DO + 2 * TILE;       // K ring (pairs)
+  static constexpr int OFF_V = OFF_K + KS * PAIR;       // V ring (pairs)
+  static constexpr int OFF_STAGE = OFF_V + VS * PAIR;   // output staging
   static constexpr int OFF_STAT = OFF_STAGE + TILE;     // statistics [2][128] fp32
   static constexpr int BYTES = OFF_STAT + 2 * 512;
   static constexpr int SMEM = BYTES + 1024;
 };
-// dQ kernel tensor memory: two fp32 S and two fp32 dP buffers (64 columns
-// each; step j uses buffer j % 2, read by the elementwise group j % 2), four
-// bf16 dS buffers (32 columns; step j uses j % 4) and the dQ accumulator.
-// The S and dP buffers are free as soon as the elementwise warps have read
-// them, so S(j + 2) does not wait for the dQ product of step j; only the dS
-// buffers wait for it, four steps later.
-constexpr int kNb = 2;   // S / dP buffers
-constexpr int kNds = 4;  // dS buffers
+// A pair tile holds, per 64-channel group h (at h * 2 * 8192), the first
+// cube's 64 rows and then the second's, 128 B each in the 128-byte swizzle:
+// one 128-row K-major operand (S, dP) or one 128-key MN-major operand (dQ).
+//
+// dQ kernel tensor memory: one fp32 S and one fp32 dP buffer (128 columns
+// each), released as soon as the elementwise warps have read them; two bf16
+// dS buffers (64 packed columns; step j uses j % 2), released by the dQ
+// product; the dQ accumulator (D columns).
 constexpr uint32_t kQS = 0, kQP = 128, kQdS = 256, kQAcc = 384;
 
 struct __align__(8) DqBars {
-  uint64_t k_full[8], k_empty[8], v_full[8], v_empty[8];  // rings of DqL<D>::KS / VS slots
+  uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];  // rings of DqL<D>::KS / VS slots
   uint64_t q_full[2], q_empty[2];
-  uint64_t s_full[kNb], dp_full[kNb], s_free[kNb], dp_free[kNb];
-  uint64_t ds_full[kNds], ds_free[kNds];
+  uint64_t s_full, dp_full, s_free, dp_free;
+  uint64_t ds_full[2], ds_free[2];
   uint64_t acc_full, acc_empty;
   uint64_t drain[3];
 };
+
 struct alignas(16) DqShared {
   DqBars bar;
   uint32_t tmem_base;
@@ -281,14 +289,12 @@ __global__ void __launch_bounds__(kThreads, 1) fine_dq_kernel(const __grid_const
     for (int i = 0; i < L::KS; ++i) { mbar_init(&B.k_full[i], 1); mbar_init(&B.k_empty[i], 1); }
     for (int i = 0; i < L::VS; ++i) { mbar_init(&B.v_full[i], 1); mbar_init(&B.v_empty[i], 1); }
     for (int i = 0; i < 2; ++i) { mbar_init(&B.q_full[i], 1); mbar_init(&B.q_empty[i], 2 + 8); }
-    for (int b = 0; b < kNb; ++b) {
-      mbar_init(&B.s_full[b], 1);
-      mbar_init(&B.dp_full[b], 1);
-      mbar_init(&B.s_free[b], 4);
-      mbar_init(&B.dp_free[b], 4);
-    }
-    for (int d = 0; d < kNds; ++d) {
-      mbar_init(&B.ds_full[d], 4);
+    mbar_init(&B.s_full, 1);
+    mbar_init(&B.dp_full, 1);
+    mbar_init(&B.s_free, 8);
+    mbar_init(&B.dp_free, 8);
+    for (int d = 0; d < 2; ++d) {
+      mbar_init(&B.ds_full[d], 8);
       mbar_init(&B.ds_free[d], 1);
     }
     mbar_init(&B.acc_full, 1);
@@ -333,19 +339,28 @@ __global__ void __launch_bounds__(kThreads, 1) fine_dq_kernel(const __grid_const
         }
         bulk_load(tiles + L::OFF_STAT + qb * 512, p.qstat + (size_t)c.item * 128, 512, &B.q_full[qb]);
         ++gq;
-        for (int t = 0; t < c.n; ++t) {
-          int j = p.list[(size_t)c.item * p.kcap + t];
-          if (j < 0 || j >= C) { bad = true; j = 0; }
-          const size_t row = ((size_t)bh * C + j) * 64;
+        const int steps = (c.n + 1) >> 1;
+        for (int t = 0; t < steps; ++t) {
+          int ja = p.list[(size_t)c.item * p.kcap + 2 * t];
+          int jb = 2 * t + 1 < c.n ? p.list[(size_t)c.item * p.kcap + 2 * t + 1] : ja;  // odd tail: a copy
+          if (ja < 0 || ja >= C) { bad = true; ja = 0; }
+          if (jb < 0 || jb >= C) { bad = true; jb = 0; }
+          const int ra = (bh * C + ja) * 64, rb = (bh * C + jb) * 64;
           const int ks = gk % L::KS, vs = gk % L::VS;
           if (gk >= L::KS && !W.wait(&B.k_empty[ks], ((gk / L::KS) - 1) & 1)) { aborted = true; break; }
-          mbar_arrive_expect_tx(&B.k_full[ks], L::TILE);
-          for (int h = 0; h < L::NH; ++h)
-            tma_load_2d(tiles + L::OFF_K + ks * L::TILE + h * 8192, &p.tm_k, &B.k_full[ks], 64 * h, (int)row);
+          mbar_arrive_expect_tx(&B.k_full[ks], L::PAIR);
+          uint8_t* kd = tiles + L::OFF_K + ks * L::PAIR;
+          for (int h = 0; h < L::NH; ++h) {
+            tma_load_2d(kd + h * 16384, &p.tm_k, &B.k_full[ks], 64 * h, ra);
+            tma_load_2d(kd + h * 16384 + 8192, &p.tm_k, &B.k_full[ks], 64 * h, rb);
+          }
           if (gk >= L::VS && !W.wait(&B.v_empty[vs], ((gk / L::VS) - 1) & 1)) { aborted = true; break; }
-          mbar_arrive_expect_tx(&B.v_full[vs], L::TILE);
-          for (int h = 0; h < L::NH; ++h)
-            tma_load_2d(tiles + L::OFF_V + vs * L::TILE + h * 8192, &p.tm_v, &B.v_full[vs], 64 * h, (int)row);
+          mbar_arrive_expect_tx(&B.v_full[vs], L::PAIR);
+          uint8_t* vd = tiles + L::OFF_V + vs * L::PAIR;
+          for (int h = 0; h < L::NH; ++h) {
+            tma_load_2d(vd + h * 16384, &p.tm_v, &B.v_full[vs], 64 * h, ra);
+            tma_load_2d(vd + h * 16384 + 8192, &p.tm_v, &B.v_full[vs], 64 * h, rb);
+          }
           ++gk;
         }
         if (aborted) break;
@@ -363,39 +378,41 @@ __global__ void __launch_bounds__(kThreads, 1) fine_dq_kernel(const __grid_const
     regs_dec<56>();
     if (lane == 0) {
       const bool is_s = warp == 1;
-      constexpr uint32_t idesc = idesc_bf16_f32(64, 64, false, false);
-      const uint32_t col0 = is_s ? kQS : kQP;
+      constexpr uint32_t idesc = idesc_bf16_f32(64, 128, false, false);
+      const uint32_t col = is_s ? kQS : kQP;
       const int ring = is_s ? L::KS : L::VS;
       const uint64_t adesc0 = sdesc_sw128(smem_u32(tiles + (is_s ? L::OFF_Q : L::OFF_DO)), 16, 1024);
       const uint64_t bdesc0 = sdesc_sw128(smem_u32(tiles + (is_s ? L::OFF_K : L::OFF_V)), 16, 1024);
       uint64_t* full = is_s ? B.k_full : B.v_full;
-      uint64_t* freed = is_s ? B.s_free : B.dp_free;
-      uint64_t* done = is_s ? B.s_full : B.dp_full;
+      uint64_t* freed = is_s ? &B.s_free : &B.dp_free;
+      uint64_t* done = is_s ? &B.s_full : &B.dp_full;
       bool aborted = false, issued = false;
-      int j = 0, b = 0, u = 0;
+      int j = 0;  // CTA step
       Cur c;
       cur_init<false>(p, c);
       while (c.live && !aborted) {
         const int qb = c.is & 1;
-        for (int t = 0; t < c.n; ++t) {
+        const int steps = (c.n + 1) >> 1;
+        for (int t = 0; t < steps; ++t) {
           const int rs = j % ring;
-          if ((u >= 1 && !W.wait(&freed[b], (u - 1) & 1)) ||
-              (t == 0 && !W.wait(&B.q_full[qb], (c.is >> 1) & 1)) || !W.wait(&full[rs], (j / ring) & 1)) {
+          // The single S (dP) buffer is free once the elementwise warps have read step j - 1.
+          if ((j >= 1 && !W.wait(freed, (j - 1) & 1)) || (t == 0 && !W.wait(&B.q_full[qb], (c.is >> 1) & 1)) ||
+              !W.wait(&full[rs], (j / ring) & 1)) {
             aborted = true;
             break;
           }
           tc_fence_after();
           const uint64_t ad = adesc0 + (uint64_t)((qb * L::TILE) >> 4);
-          const uint64_t bd = bdesc0 + (uint64_t)((rs * L::TILE) >> 4);
+          const uint64_t bd = bdesc0 + (uint64_t)((rs * L::PAIR) >> 4);
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k)
-            mma_bf16_ss(tmem + col0 + 64u * b, ad + kmajor_off(k), bd + kmajor_off(k), idesc, k > 0 ? 1u : 0u);
-          mma_commit(&done[b]);
+          for (int k = 0; k < D / 16; ++k)  // steps of 16 along D
+            mma_bf16_ss(tmem + col, ad + kmajor_off(k), bd + (uint64_t)(((k >> 2) * 16384 + (k & 3) * 32) >> 4),
+                        idesc, k > 0 ? 1u : 0u);
+          mma_commit(done);
           if (!is_s) mma_commit(&B.v_empty[rs]);
-          if (t == c.n - 1) mma_commit(&B.q_empty[qb]);
+          if (t == steps - 1) mma_commit(&B.q_empty[qb]);
           issued = true;
           ++j;
-          if (++b == kNb) { b = 0; ++u; }
         }
         if (aborted) break;
         cur_next_item<false>(p, c);
@@ -411,30 +428,31 @@ __global__ void __launch_bounds__(kThreads, 1) fine_dq_kernel(const __grid_const
     regs_dec<56>();
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(64, D, false, true);
-      const uint64_t kdesc0 = sdesc_sw128(smem_u32(tiles + L::OFF_K), 8192, 1024);  // MN-major K
+      const uint64_t kdesc0 = sdesc_sw128(smem_u32(tiles + L::OFF_K), 16384, 1024);  // MN-major K pair
       bool aborted = false, issued = false;
-      int j = 0, d = 0, ud = 0;  // CTA step, its dS buffer and use count
+      int j = 0;  // CTA step; dS buffer j % 2, its use j / 2
       Cur c;
       cur_init<false>(p, c);
       while (c.live && !aborted) {
-        for (int t = 0; t < c.n; ++t) {
-          const int ks = j % L::KS;
-          if ((t == 0 && c.is >= 1 && !W.wait(&B.acc_empty, (c.is - 1) & 1)) || !W.wait(&B.ds_full[d], ud & 1)) {
+        const int steps = (c.n + 1) >> 1;
+        for (int t = 0; t < steps; ++t) {
+          const int ks = j % L::KS, d = j & 1;
+          if ((t == 0 && c.is >= 1 && !W.wait(&B.acc_empty, (c.is - 1) & 1)) ||
+              !W.wait(&B.ds_full[d], (j >> 1) & 1)) {
             aborted = true;
             break;
           }
           tc_fence_after();
-          const uint64_t kd = kdesc0 + (uint64_t)((ks * L::TILE) >> 4);
+          const uint64_t kd = kdesc0 + (uint64_t)((ks * L::PAIR) >> 4);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma_bf16_ts(tmem + kQAcc, tmem + kQdS + 32u * d + packed_col(k), kd + (uint64_t)((k * 2048) >> 4), idesc,
+          for (int k = 0; k < 8; ++k)  // 8 slices of 16 keys
+            mma_bf16_ts(tmem + kQAcc, tmem + kQdS + 64u * d + packed_col(k), kd + (uint64_t)((k * 2048) >> 4), idesc,
                         (t > 0 || k > 0) ? 1u : 0u);
           mma_commit(&B.ds_free[d]);
           mma_commit(&B.k_empty[ks]);
-          if (t == c.n - 1) mma_commit(&B.acc_full);
+          if (t == steps - 1) mma_commit(&B.acc_full);
           issued = true;
           ++j;
-          if (++d == kNds) { d = 0; ++ud; }
         }
         if (aborted) break;
         cur_next_item<false>(p, c);
@@ -447,12 +465,11 @@ __global__ void __launch_bounds__(kThreads, 1) fine_dq_kernel(const __grid_const
     __syncwarp();
   } else if (warp < 12) {
     // ------------------------------------------------------------ P, dS
-    // Group grp takes the steps j with j % 2 == grp, i.e. S / dP buffer grp.
-    const int quarter = warp & 3, grp = (warp - 4) >> 2;
+    // Warp w: lane quarter w % 4 (rows), key half (w - 4) / 4 of every step.
+    const int quarter = warp & 3, hf = (warp - 4) >> 2;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const int ra = quarter * 16 + (lane >> 2);
     const float sl2 = p.scale_log2;
-    const int b = grp;
     int j = 0;  // CTA step
     Cur c;
     cur_init<false>(p, c);
@@ -463,29 +480,33 @@ __global__ void __launch_bounds__(kThreads, 1) fine_dq_kernel(const __grid_const
       const float l0 = stat[ra], l1 = stat[ra + 8], d0 = stat[64 + ra], d1 = stat[64 + ra + 8];
       __syncwarp();
       if (lane == 0) mbar_arrive(&B.q_empty[qb]);
-      for (int t = 0; t < c.n; ++t, ++j) {
-        if ((j & 1) != grp) continue;
-        const int u = j >> 1;                  // use of S / dP buffer b
-        const int d = j % kNds, ud = j / kNds;  // dS buffer and its use
-        W.wait(&B.s_full[b], u & 1);
-        W.wait(&B.dp_full[b], u & 1);
+      const int steps = (c.n + 1) >> 1;
+      for (int t = 0; t < steps; ++t, ++j) {
+        const int d = j & 1, ud = j >> 1;  // dS buffer and its use
+        W.wait(&B.s_full, j & 1);
+        W.wait(&B.dp_full, j & 1);
         tc_fence_after();
         uint32_t sr[32], g[32];
-        tmem_ld16x256b_x8(tmem + lane_base + kQS + 64u * b, sr);
-        tmem_ld16x256b_x8(tmem + lane_base + kQP + 64u * b, g);
+        tmem_ld16x256b_x8(tmem + lane_base + kQS + 64u * hf, sr);
+        tmem_ld16x256b_x8(tmem + lane_base + kQP + 64u * hf, g);
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&B.s_free[b]);
-          mbar_arrive(&B.dp_free[b]);
+          mbar_arrive(&B.s_free);
+          mbar_arrive(&B.dp_free);
         }
         uint32_t pk_p[16], pk_s[16];
         p_ds<true>(sr, g, sl2, l0, l1, d0, d1, nullptr, nullptr, 0, pk_p, pk_s);
-        // dS buffer d is free once the dQ product of step j - 4 completed
+        if (hf == 1 && 2 * t + 1 >= c.n) {
+          // odd tail: keys 64..127 repeat the last cube and do not take part
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk_s[e] = 0u;
+        }
+        // dS buffer d is free once the dQ product of step j - 2 completed
         if (ud >= 1) W.wait(&B.ds_free[d], (ud - 1) & 1);
         tc_fence_after();
-        tmem_st16x128b_x8(tmem + lane_base + kQdS + 32u * d, pk_s);
+        tmem_st16x128b_x8(tmem + lane_base + kQdS + 64u * d + 32u * hf, pk_s);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
