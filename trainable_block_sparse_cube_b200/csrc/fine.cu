@@ -47,7 +47,9 @@
 //   warp 2      issuer of the S MMAs (also allocates tensor memory)
 //   warp 3      issuer of the O MMAs
 //   warps 4-11  softmax
-//   warps 12-15 epilogue: Q loads, gates and coarse rows, output tiles (TMA)
+//   warps 12-15 epilogue: Q loads (item is + 2 into the buffer of item is as
+//               soon as item is's S products completed), gates and coarse
+//               rows, output tiles (TMA)
 //
 // Every mbarrier wait is bounded (plan wait limit). A wait that gives up
 // records kErrTimeout, sets a CTA-wide abort flag that makes every later wait
@@ -198,6 +200,8 @@ struct __align__(8) Bars {
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t q_full[2];     // Q of item is in smem buffer is % 2 (TMA)
+  uint64_t q_free[2];     // S issuer -> epilogue: every S product of item is complete (commit)
+  uint64_t lp_free[2];    // epilogue -> softmax: row statistics of item is read (count 4)
   uint64_t s_full[kSP];   // S issuer -> softmax: S of step j in buffer j % 3 (commit)
   uint64_t p_full[kSP];   // softmax -> O issuer: P of step j in buffer j % 3 (count 8)
   uint64_t sp_free[kSP];  // O issuer -> S issuer, softmax: O of step j complete (commit)
@@ -352,6 +356,8 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
       mbar_init(&B.q_full[b], 1);
       mbar_init(&B.l_full[b], 8);
       mbar_init(&B.drain[b], 1);
+      mbar_init(&B.q_free[b], 1);
+      mbar_init(&B.lp_free[b], 4);
     }
     mbar_init(&B.o_full, 1);
     mbar_init(&B.o_empty, 4);
@@ -468,6 +474,8 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
                       kd + (uint64_t)(((k >> 2) * 16384 + (k & 3) * 32) >> 4), idesc_s, k > 0 ? 1u : 0u);
         mma_commit(&B.k_empty[ks]);
         mma_commit(&B.s_full[b]);
+        // The item's last S product: once it completes, its Q buffer is free.
+        if (c.t == c.ntiles - 1) mma_commit(&B.q_free[c.is & 1]);
         issued_any = true;
         ++j;
         if (++b == kSP) { b = 0; ++u; }
@@ -596,7 +604,9 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
         if (lane == 0) mbar_arrive(&B.p_full[b]);
         if (++b == kSP) { b = 0; ++u; }
       }
-      // Row sums of the item (this key half) -> the epilogue.
+      // Row sums of the item (this key half) -> the epilogue, once it has read
+      // those of the item two back (the same entries).
+      if (c.is >= 2) W.wait(&B.lp_free[ob], ((c.is >> 1) - 1) & 1);
       l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
       l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
       l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
@@ -670,6 +680,11 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
       const int bh = item / C, ci = item - bh * C;
       const int ct = ci / (Hc * Wc), ch = (ci / Wc) % Hc, cw = ci % Wc;
       const int ob = is & 1;
+      // Q of item is + 2 goes into this item's buffer as soon as the item's
+      // S products have completed, not after its O read-out: the 5-D raster
+      // box from HBM then has most of an item to land (waiting for the O
+      // read-out left the S issuer stalled on Q at item boundaries).
+      if (item_at(p, is + 2) >= 0 && (est != 0 || W.wait(&B.q_free[ob], (is >> 1) & 1))) load_q(is + 2);
       prefetch(is + 1);
       W.wait(&B.l_full[ob], (is >> 1) & 1);
       const float lsum0 = sh.lpart[ob][0][ra] + sh.lpart[ob][1][ra];
@@ -682,6 +697,8 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
         p.lse[(size_t)bh * p.N + tok_of(ra)] = 0.6931471805599453f * (sh.mref[ob][ra] + __log2f(lsum0));
         p.lse[(size_t)bh * p.N + tok_of(ra + 8)] = 0.6931471805599453f * (sh.mref[ob][ra + 8] + __log2f(lsum1));
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&B.lp_free[ob]);  // row statistics of item is read
       W.wait(&B.o_full, is & 1);
       tc_fence_after();
       float o[2 * D / 4];
@@ -696,8 +713,6 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&B.o_empty);
-      // All S steps of this item completed: its Q buffer takes item is + 2.
-      load_q(is + 2);
       cp_async_wait<1>();               // this item's gates and coarse row (older group) landed
       if (est == 0) bulk_wait_read0();  // the previous item's output stores have read the staging tile
       epi_sync();
