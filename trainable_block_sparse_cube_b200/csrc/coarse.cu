@@ -16,14 +16,17 @@
 // dropped ones are below 2^-24 relative.
 //   1. scores   s = qbar kbar^T / sqrt(D)       [BH, C, C]   (tcgen05, 128 x 128 tiles)
 //   2. select   one warp per row, the row's scores as order-preserving
-//               uint32 keys in shared memory: row max and sum, the
-//               probabilities P written as bf16 terms (hi and mid for the
-//               forward's output product, also lo when the backward's
-//               products need them), then the selection. Top-K <= 32: the minimum of the lanes' maxima
-//               bounds the K-th largest key from below, the keys at or above
-//               it are compacted in place (ascending id) and an MSB-first
-//               count search over them finds the K-th largest; larger K, or
-//               more than 256 candidates, search over all keys. Top-p (own
+//               uint32 keys: row max and sum, the probabilities P written as
+//               bf16 terms (hi and mid for the forward's output product, also
+//               lo when the backward's products need them), then the
+//               selection. Top-K <= 32 with C <= 1024 (own kernel): the row
+//               stays in registers; the minimum of the lanes' maxima bounds
+//               the K-th largest key from below, each lane places its keys at
+//               or above it through a prefix sum over the lanes, an MSB-first
+//               count search over those candidates finds the K-th largest,
+//               and the ids go out through two bitmaps (above it, equal to it)
+//               in ascending order. Larger K or C, or more than 256
+//               candidates, search over all keys in shared memory. Top-p (own
 //               kernel): the exact kmax-th largest key by the same search,
 //               the kmax candidates ranked by (score desc, id asc) and cut at
 //               the first prefix whose mass reaches p, clamped to
@@ -127,36 +130,35 @@ __device__ __forceinline__ void row_softmax(const CoarseParams& p, int row, uint
   }
 }
 
-// row_softmax for C <= 1024 with the row in registers: lane t holds columns
-// 64u + 2t and 64u + 2t + 1 (u < C/64 rounded up), so every score is read
-// once, every exponential computed once, and the probabilities' three terms
-// are stored as bf16 pairs. The keys still go to shared memory for the
-// selection.
-__device__ __forceinline__ void row_softmax_regs(const CoarseParams& p, int row, uint32_t* keys, int lane, float& mb,
-                                                 float& l, uint32_t& lkmax) {
+// Row `row` of the scores in registers for C <= 1024: lane t holds columns
+// 64u + 2t and 64u + 2t + 1 (u < 16) in v[2u], v[2u + 1]; -inf past C.
+__device__ __forceinline__ void load_row_regs(const CoarseParams& p, int row, int lane, float (&v)[32]) {
   const int C = p.C;
   const float* srow = p.s + (size_t)row * C;
-  float v[32];
-  float lm = -INFINITY;
-  lkmax = 0;
+  if ((C & 1) == 0) {  // even C: every row starts 8-byte aligned and a pair never straddles C
 #pragma unroll
-  for (int u = 0; u < 16; ++u) {
-    const int j = 64 * u + 2 * lane;
-    v[2 * u] = j < C ? srow[j] : -INFINITY;
-    v[2 * u + 1] = j + 1 < C ? srow[j + 1] : -INFINITY;
+    for (int u = 0; u < 16; ++u) {
+      const int j = 64 * u + 2 * lane;
+      const float2 x = j < C ? *reinterpret_cast<const float2*>(srow + j) : make_float2(-INFINITY, -INFINITY);
+      v[2 * u] = x.x;
+      v[2 * u + 1] = x.y;
+    }
+  } else {
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int j = 64 * u + 2 * lane;
+      v[2 * u] = j < C ? srow[j] : -INFINITY;
+      v[2 * u + 1] = j + 1 < C ? srow[j + 1] : -INFINITY;
+    }
   }
-#pragma unroll
-  for (int u = 0; u < 16; ++u) {
-    const int j = 64 * u + 2 * lane;
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-      if (j + h < C) {
-        const uint32_t k = order_key(v[2 * u + h]);
-        keys[j + h] = k;
-        lkmax = max(lkmax, k);
-        lm = fmaxf(lm, v[2 * u + h]);
-      }
-  }
+}
+
+// Softmax of a register-resident row (load_row_regs layout) with row max lm:
+// writes the probabilities' terms as bf16 pairs, returns the row max in log2
+// units (mb) and the row sum l. v is overwritten with the numerators.
+__device__ __forceinline__ void softmax_store_regs(const CoarseParams& p, int row, int lane, float (&v)[32], float lm,
+                                                   float& mb, float& l) {
+  const int C = p.C;
   mb = warp_max(lm) * kLog2e;
   float ls = 0.f;
 #pragma unroll
@@ -184,6 +186,31 @@ __device__ __forceinline__ void row_softmax_regs(const CoarseParams& p, int row,
       }
     }
   }
+}
+
+// row_softmax for C <= 1024 with the row in registers, so every score is read
+// once and every exponential computed once; the keys still go to shared
+// memory for the selection.
+__device__ __forceinline__ void row_softmax_regs(const CoarseParams& p, int row, uint32_t* keys, int lane, float& mb,
+                                                 float& l, uint32_t& lkmax) {
+  const int C = p.C;
+  float v[32];
+  load_row_regs(p, row, lane, v);
+  float lm = -INFINITY;
+  lkmax = 0;
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    const int j = 64 * u + 2 * lane;
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      if (j + h < C) {
+        const uint32_t k = order_key(v[2 * u + h]);
+        keys[j + h] = k;
+        lkmax = max(lkmax, k);
+        lm = fmaxf(lm, v[2 * u + h]);
+      }
+  }
+  softmax_store_regs(p, row, lane, v, lm, mb, l);
   __syncwarp();
 }
 
@@ -235,6 +262,158 @@ __device__ __forceinline__ void topk_from_candidates(const uint32_t* ckey, const
   }
 }
 
+// Warp-wide inclusive prefix sum.
+__device__ __forceinline__ int warp_incl_scan(int x, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  return x;
+}
+
+// Top-K emission for Kt <= 32 and C <= 1024 from candidates in any order
+// (keys at or above the lower bound lo with their ids, NS slots per lane):
+// the Kt-th largest key T by the MSB-first search below the bits that lo and
+// the row maximum hi share, then the ids through two 32-word bitmaps in
+// shared memory (bm[0..31]: keys above T, bm[32..63]: keys equal to T). Word
+// w holds ids 32w..32w+31, so lane w emits its word's ids in ascending order
+// at the prefix of the words before it, and the ties taken are the lowest ids.
+template <int NS>
+__device__ __forceinline__ void topk_bitmap_emit(const uint32_t* ckey, const int* cidx, int n, int Kt, uint32_t lo,
+                                                 uint32_t hi, uint32_t* bm, int32_t* irow) {
+  const int lane = threadIdx.x & 31;
+  uint32_t ck[NS];
+  int cj[NS];
+#pragma unroll
+  for (int i = 0; i < NS; ++i) {
+    const int e = lane + 32 * i;
+    ck[i] = e < n ? ckey[e] : 0u;
+    cj[i] = e < n ? cidx[e] : 0;
+  }
+  uint32_t T = lo;
+  if (lo != hi) {
+    const int hb = 31 - __clz(lo ^ hi);
+    T = hi & ~((2u << hb) - 1u);
+    for (int b = hb; b >= 0; --b) {
+      const uint32_t c = T | (1u << b);
+      unsigned cnt = 0;
+#pragma unroll
+      for (int i = 0; i < NS; ++i) cnt += (ck[i] >= c);
+      if ((int)__reduce_add_sync(0xffffffffu, cnt) >= Kt) T = c;
+    }
+  }
+  bm[lane] = 0u;
+  bm[32 + lane] = 0u;
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < NS; ++i)
+    if (lane + 32 * i < n && ck[i] >= T) atomicOr(&bm[(ck[i] > T ? 0 : 32) + (cj[i] >> 5)], 1u << (cj[i] & 31));
+  __syncwarp();
+  const uint32_t g = bm[lane], q = bm[32 + lane];
+  const int need = Kt - (int)__reduce_add_sync(0xffffffffu, (unsigned)__popc(g));
+  const int neq = __popc(q);
+  int take = min(max(need - (warp_incl_scan(neq, lane) - neq), 0), neq);
+  uint32_t sel = g, rest = q;
+  for (; take > 0; --take) {
+    sel |= rest & (0u - rest);  // lowest remaining tie
+    rest &= rest - 1u;
+  }
+  const int c = __popc(sel);
+  int pos = warp_incl_scan(c, lane) - c;
+  while (sel) {
+    irow[pos++] = 32 * lane + (__ffs(sel) - 1);
+    sel &= sel - 1u;
+  }
+}
+
+// Ids of the Kt largest of the row's C keys (in shared memory, any Kt), ties
+// to the lower id, ascending: the Kt-th largest key by the bit search over
+// all keys, then the ids above it and the lowest-id ones equal to it.
+__device__ __forceinline__ void topk_full_search(const uint32_t* keys, int C, int Kt, int lane, int32_t* irow) {
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  const uint32_t T = kth_largest(keys, C, Kt, lane);
+  unsigned gt = 0;
+  for (int j = lane; j < C; j += 32) gt += (keys[j] > T);
+  const int need = Kt - (int)__reduce_add_sync(0xffffffffu, gt);
+  int pos = 0, eq_seen = 0;
+  for (int j0 = 0; j0 < C; j0 += 32) {
+    const int j = j0 + lane;
+    const uint32_t k = j < C ? keys[j] : 0u;
+    const bool is_eq = j < C && k == T;
+    const unsigned eqb = __ballot_sync(0xffffffffu, is_eq);
+    const bool take = (j < C && k > T) || (is_eq && eq_seen + __popc(eqb & lt_mask) < need);
+    const unsigned tb = __ballot_sync(0xffffffffu, take);
+    if (take) irow[pos + __popc(tb & lt_mask)] = j;
+    pos += __popc(tb);
+    eq_seen += __popc(eqb);
+  }
+}
+
+// Top-K for Kt <= 32 and C <= 1024 with the row in registers. The minimum of
+// the lanes' maxima bounds the Kt-th largest key from below (every lane holds
+// at least one key when C >= 64; below that a lane without keys contributes
+// 0, so every key is a candidate). Each lane counts its keys at or above the
+// bound, a prefix sum over the lanes places them, and they are written to
+// shared memory with their ids before the exponentials overwrite the row; the
+// selection then runs over the candidates alone. More than kCandCap
+// candidates (e.g. many equal scores) fall back to all keys in shared memory
+// and the full search.
+__device__ __forceinline__ void select_topk_regs(const CoarseParams& p, int row, uint32_t* keys, int* cidx,
+                                                 uint32_t* bm, int lane) {
+  const int C = p.C, Kt = p.topk;
+  float v[32];
+  load_row_regs(p, row, lane, v);
+  // The row as keys, in place (the key map is a bijection: key_value undoes it
+  // exactly, -inf padding included), so only one copy of the row is live.
+  uint32_t lkmax = 0;
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    const uint32_t k = order_key(v[e]);
+    v[e] = __uint_as_float(k);
+    if (64 * (e >> 1) + 2 * lane + (e & 1) < C) lkmax = max(lkmax, k);
+  }
+  const uint32_t lo = __reduce_min_sync(0xffffffffu, lkmax);
+  const uint32_t hi = __reduce_max_sync(0xffffffffu, lkmax);
+  int nl = 0;
+#pragma unroll
+  for (int e = 0; e < 32; ++e)
+    nl += (64 * (e >> 1) + 2 * lane + (e & 1) < C && __float_as_uint(v[e]) >= lo) ? 1 : 0;
+  const int incl = warp_incl_scan(nl, lane);
+  const int n = __shfl_sync(0xffffffffu, incl, 31);
+  if (n <= kCandCap) {
+    int pos = incl - nl;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const int j = 64 * (e >> 1) + 2 * lane + (e & 1);
+      const uint32_t k = __float_as_uint(v[e]);
+      if (j < C && k >= lo) {
+        keys[pos] = k;
+        cidx[pos] = j;
+        ++pos;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const int j = 64 * (e >> 1) + 2 * lane + (e & 1);
+      if (j < C) keys[j] = __float_as_uint(v[e]);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 32; ++e) v[e] = key_value(__float_as_uint(v[e]));
+  float mb, l;
+  softmax_store_regs(p, row, lane, v, key_value(hi), mb, l);
+  __syncwarp();
+  int32_t* irow = p.idx + (size_t)row * p.kcap;
+  if (n <= 32) topk_bitmap_emit<1>(keys, cidx, n, Kt, lo, hi, bm, irow);
+  else if (n <= 64) topk_bitmap_emit<2>(keys, cidx, n, Kt, lo, hi, bm, irow);
+  else if (n <= 128) topk_bitmap_emit<4>(keys, cidx, n, Kt, lo, hi, bm, irow);
+  else if (n <= kCandCap) topk_bitmap_emit<8>(keys, cidx, n, Kt, lo, hi, bm, irow);
+  else topk_full_search(keys, C, Kt, lane, irow);
+  if (lane == 0) p.cnt[row] = Kt;
+}
+
 // Fixed top-K (any K), and the probabilities alone when the selection is
 // supplied by the caller, with the row's keys in shared memory instead of
 // registers, so more warps (rows) per SM hide the latency of the warp-wide
@@ -253,7 +432,7 @@ __global__ void __launch_bounds__(256, 4) coarse_select_topk_kernel(const Coarse
   if (row >= p.BH * p.C) return;
   const int C = p.C, Kt = p.topk;
   const int stride = (C + 31) / 32 * 32;
-  uint32_t* keys = reinterpret_cast<uint32_t*>(dyn) + (size_t)warp * (stride + kCandCap);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(dyn) + (size_t)warp * (stride + kCandCap + 64);
   int* cidx = reinterpret_cast<int*>(keys + stride);
   const uint32_t lt_mask = (1u << lane) - 1u;
   float mb, l;
@@ -294,26 +473,23 @@ __global__ void __launch_bounds__(256, 4) coarse_select_topk_kernel(const Coarse
     else if (n <= 128) topk_from_candidates<4>(keys, cidx, n, Kt, lo, hi, irow);
     else topk_from_candidates<8>(keys, cidx, n, Kt, lo, hi, irow);
   } else {
-    // Bit search for the Kt-th largest key over all keys, then the ids above it
-    // and the lowest-id ones equal to it, ascending.
-    const uint32_t T = kth_largest(keys, C, Kt, lane);
-    unsigned gt = 0;
-    for (int j = lane; j < C; j += 32) gt += (keys[j] > T);
-    const int need = Kt - (int)__reduce_add_sync(0xffffffffu, gt);
-    int pos = 0, eq_seen = 0;
-    for (int j0 = 0; j0 < C; j0 += 32) {
-      const int j = j0 + lane;
-      const uint32_t k = j < C ? keys[j] : 0u;
-      const bool is_eq = j < C && k == T;
-      const unsigned eqb = __ballot_sync(0xffffffffu, is_eq);
-      const bool take = (j < C && k > T) || (is_eq && eq_seen + __popc(eqb & lt_mask) < need);
-      const unsigned tb = __ballot_sync(0xffffffffu, take);
-      if (take) irow[pos + __popc(tb & lt_mask)] = j;
-      pos += __popc(tb);
-      eq_seen += __popc(eqb);
-    }
+    topk_full_search(keys, C, Kt, lane, irow);
   }
   if (lane == 0) p.cnt[row] = Kt;
+}
+
+// Top-K for Kt <= 32 and C <= 1024 (select_topk_regs), one warp per row;
+// per warp the shared memory holds the candidates' keys (C rounded up to 32),
+// kCandCap candidate ids and the two emission bitmaps.
+__global__ void __launch_bounds__(256, 3) coarse_select_topk_regs_kernel(const CoarseParams p) {
+  extern __shared__ __align__(16) uint8_t dyn[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 8 + warp;
+  if (row >= p.BH * p.C) return;
+  const int stride = (p.C + 31) / 32 * 32;
+  uint32_t* keys = reinterpret_cast<uint32_t*>(dyn) + (size_t)warp * (stride + kCandCap + 64);
+  int* cidx = reinterpret_cast<int*>(keys + stride);
+  select_topk_regs(p, row, keys, cidx, reinterpret_cast<uint32_t*>(cidx + kCandCap), lane);
 }
 
 // Top-p selection with the row's keys in shared memory: the kmax best
@@ -592,7 +768,7 @@ cudaError_t launch_tc(const CoarseParams& p, cudaStream_t st) {
 
 cudaError_t launch_select_topk(const CoarseParams& p, cudaStream_t st) {
   const int rows = p.BH * p.C;
-  const size_t smem = (size_t)8 * ((p.C + 31) / 32 * 32 + kCandCap) * 4;
+  const size_t smem = (size_t)8 * ((p.C + 31) / 32 * 32 + kCandCap + 64) * 4;
   if (smem > 48 * 1024) {
     cudaError_t e = p.C <= 1024 ? cudaFuncSetAttribute(coarse_select_topk_kernel<true>,
                                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
@@ -600,7 +776,14 @@ cudaError_t launch_select_topk(const CoarseParams& p, cudaStream_t st) {
                                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  if (p.C <= 1024)
+  if (p.C <= 1024 && p.topk <= 32 && p.do_select) {
+    if (smem > 48 * 1024) {
+      cudaError_t e = cudaFuncSetAttribute(coarse_select_topk_regs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)smem);
+      if (e != cudaSuccess) return e;
+    }
+    coarse_select_topk_regs_kernel<<<(rows + 7) / 8, 256, smem, st>>>(p);
+  } else if (p.C <= 1024)
     coarse_select_topk_kernel<true><<<(rows + 7) / 8, 256, smem, st>>>(p);
   else
     coarse_select_topk_kernel<false><<<(rows + 7) / 8, 256, smem, st>>>(p);
