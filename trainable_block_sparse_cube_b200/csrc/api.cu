@@ -38,8 +38,6 @@ struct vsa_plan_s {
   int BH, N, C, kcap;
   char* ws;
   vsa_workspace_layout_t lay;
-  CUtensorMap tm_q;         // raster map of q, encoded for the pointer tm_q_for
-  const void* tm_q_for;
   CUtensorMap tm_k, tm_v;   // maps over the cube-major copies in the workspace
   CUtensorMap tm_qc;        // map over q's cube-major copy (written by the backward pass's gather)
   CUtensorMap tm_qs, tm_ks, tm_vs, tm_ps;  // maps over the coarse operands' bf16 terms
@@ -212,7 +210,7 @@ vsa_status encode_coarse_maps(vsa_plan_s* P) {
 // 5-D map over a raster tensor [BH][T][H][W][D] bf16 (q or out): a box
 // is one cube's 4 x 4 x 4 tokens by 64 channels, laid out in shared memory as
 // 64 rows (in-cube slot order) of 128 bytes in the 128-byte swizzle.
-vsa_status encode_raster_map(CUtensorMap* m, const void* base, const vsa_config& c, int BH, bool load) {
+vsa_status encode_raster_map(CUtensorMap* m, const void* base, const vsa_config& c, int BH) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return VSA_ERR_CUDA;
   const cuuint64_t D = (cuuint64_t)c.D;
@@ -223,7 +221,7 @@ vsa_status encode_raster_map(CUtensorMap* m, const void* base, const vsa_config&
   cuuint32_t es[5] = {1, 1, 1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, es,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   load ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_NONE,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? VSA_OK : VSA_ERR_CUDA;
 }
@@ -283,15 +281,11 @@ vsa_status run_common(vsa_plan_t P, const void* q, const void* k, const void* v,
   if (vsa::launch_coarse(cp, st) != cudaSuccess) return VSA_ERR_CUDA;
 
   vsa::FineParams fp{};
-  if (P->tm_q_for != q) {
-    const vsa_status e = encode_raster_map(&P->tm_q, q, c, P->BH, true);
-    if (e != VSA_OK) return e;
-    P->tm_q_for = q;
-  }
-  fp.tm_q = P->tm_q; fp.tm_k = P->tm_k; fp.tm_v = P->tm_v;
+  fp.tm_k = P->tm_k; fp.tm_v = P->tm_v;
+  fp.q = static_cast<const __nv_bfloat16*>(q);
   if (out) {
     if (P->tm_out_for != out) {
-      const vsa_status e = encode_raster_map(&P->tm_out, out, c, P->BH, false);
+      const vsa_status e = encode_raster_map(&P->tm_out, out, c, P->BH);
       if (e != VSA_OK) return e;
       P->tm_out_for = out;
     }
@@ -455,7 +449,7 @@ vsa_status run_backward(vsa_plan_t P, void* bws, size_t bws_bytes, const void* q
   vsa_status e = VSA_OK;
   fb.tm_q = P->tm_qc; fb.tm_k = P->tm_k; fb.tm_v = P->tm_v;
   e = encode_cube_map(&fb.tm_do, bw + BL.do_cube, rows, D);
-  if (e == VSA_OK) e = encode_raster_map(&fb.tm_out0, dq, c, P->BH, false);
+  if (e == VSA_OK) e = encode_raster_map(&fb.tm_out0, dq, c, P->BH);
   if (e != VSA_OK) return e;
   fb.qstat = pp.qstat;
   fb.err = cp.err;
@@ -476,8 +470,8 @@ vsa_status run_backward(vsa_plan_t P, void* bws, size_t bws_bytes, const void* q
   const int grid = fb.n_items < P->num_sms ? fb.n_items : P->num_sms;
   if (!mark(2)) return VSA_ERR_CUDA;
   if (vsa::launch_fine_dq(fb, D, grid, st) != cudaSuccess) return VSA_ERR_CUDA;
-  e = encode_raster_map(&fb.tm_out0, dk, c, P->BH, false);
-  if (e == VSA_OK) e = encode_raster_map(&fb.tm_out1, dv, c, P->BH, false);
+  e = encode_raster_map(&fb.tm_out0, dk, c, P->BH);
+  if (e == VSA_OK) e = encode_raster_map(&fb.tm_out1, dv, c, P->BH);
   if (e != VSA_OK) return e;
   fb.list = tp.tlist; fb.cnt = tp.tcnt; fb.off = tp.toff;
   fb.cpart0 = cb.dkbar; fb.cpart1 = cb.dvbar;

@@ -13,11 +13,13 @@
 // item's selected KV cubes (128 keys):
 //   S[64 q x 128 keys] = Q . K_pair^T     tcgen05.mma M=64, N=128 (Q, K in smem)
 //   O[64 q x D]       += P . V_pair       tcgen05.mma M=64, N=D   (P in TMEM, V in smem)
-// Each query cube is read once, straight from the raster q: a 5-D TMA box of
-// 4 x 4 x 4 tokens by 64 channels lands as 64 rows in in-cube slot order. K
-// and V cubes, read about K times each from L2, come from the cube-major
-// copies (one contiguous 64 x D tile per cube), which load faster than the
-// strided raster boxes.
+// Each query cube is read once, straight from the raster q, by the epilogue
+// warps with 16-byte cp.async copies into the 128-byte-swizzled tile (64 rows
+// in in-cube slot order): the load/store path, not the TMA unit, which then
+// serves only the K/V tiles (a raster box from HBM on the TMA unit held up the
+// K/V tiles queued behind it). K and V cubes, read about K times each from L2,
+// come from the cube-major copies (one contiguous 64 x D tile per cube) as
+// 2-D TMA boxes, which load faster than strided raster boxes.
 //
 // Tensor memory holds three S/P buffers and the O accumulator: S of steps
 // j+1 and j+2 can run on the tensor core while the softmax works on step j,
@@ -47,8 +49,8 @@
 //   warp 2      issuer of the S MMAs (also allocates tensor memory)
 //   warp 3      issuer of the O MMAs
 //   warps 4-11  softmax
-//   warps 12-15 epilogue: Q loads (item is + 2 into the buffer of item is as
-//               soon as item is's S products completed), gates and coarse
+//   warps 12-15 epilogue: Q copies (item is + 2 into the buffer of item is
+//               as soon as item is's S products completed), gates and coarse
 //               rows, output tiles (TMA)
 //
 // Every mbarrier wait is bounded (plan wait limit). A wait that gives up
@@ -199,7 +201,7 @@ struct Layout {
 struct __align__(8) Bars {
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
-  uint64_t q_full[2];     // Q of item is in smem buffer is % 2 (TMA)
+  uint64_t q_full[2];     // Q of item is in smem buffer is % 2 (count 128: every epilogue thread)
   uint64_t q_free[2];     // S issuer -> epilogue: every S product of item is complete (commit)
   uint64_t lp_free[2];    // epilogue -> softmax: row statistics of item is read (count 4)
   uint64_t s_full[kSP];   // S issuer -> softmax: S of step j in buffer j % 3 (commit)
@@ -353,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
       mbar_init(&B.sp_free[b], 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&B.q_full[b], 1);
+      mbar_init(&B.q_full[b], 128);
       mbar_init(&B.l_full[b], 8);
       mbar_init(&B.drain[b], 1);
       mbar_init(&B.q_free[b], 1);
@@ -366,7 +368,6 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    prefetch_tmap(&p.tm_q);
     prefetch_tmap(&p.tm_k);
     prefetch_tmap(&p.tm_v);
     if (p.out) prefetch_tmap(&p.tm_out);
@@ -635,21 +636,32 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
     uint8_t* stage = tiles + L::OFF_STAGE;
     const int Hc = p.H >> 2, Wc = p.W >> 2;
     int qloads0 = 0, qloads1 = 0;
-    // Q of item `is` -> smem buffer is & 1 (TMA, one thread).
+    // Q of item `is` -> smem buffer is & 1: each epilogue thread copies 16-byte
+    // chunks of token rows (cp.async) to chunk c ^ (row % 8) of the row, the
+    // 128-byte swizzle of the MMA operand; the copies complete in the thread's
+    // cp.async group and are published by q_arrive (proxy fence, then one
+    // arrival per thread on q_full).
+    constexpr int CPR = D / 8, RPI = 128 / CPR;  // 16-byte chunks per token row, rows per pass
     auto load_q = [&](int is) {
       const int item = item_at(p, is);
       if (item < 0) return;
       const int b = is & 1;
       if (b == 0) ++qloads0; else ++qloads1;
-      if (est == 0) {
-        const int bh = item / C, ci = item - bh * C;
-        const int ct = ci / (Hc * Wc), ch = (ci / Wc) % Hc, cw = ci % Wc;
-        uint8_t* dst = tiles + L::OFF_Q + b * L::Q_BYTES;
-        mbar_arrive_expect_tx(&B.q_full[b], L::Q_BYTES);
+      const int bh = item / C, ci = item - bh * C;
+      const int ct = ci / (Hc * Wc), ch = (ci / Wc) % Hc, cw = ci % Wc;
+      uint8_t* dst = tiles + L::OFF_Q + b * L::Q_BYTES;
+      const int chunk = est % CPR, r0 = est / CPR, h = chunk >> 3, cc = chunk & 7;
 #pragma unroll
-        for (int h = 0; h < L::NH; ++h)
-          tma_load_5d(dst + h * 8192, &p.tm_q, &B.q_full[b], 64 * h, 4 * cw, 4 * ch, 4 * ct, bh);
+      for (int i = 0; i < 64 / RPI; ++i) {
+        const int r = r0 + RPI * i;
+        const int tok = ((4 * ct + (r >> 4)) * p.H + 4 * ch + ((r >> 2) & 3)) * p.W + 4 * cw + (r & 3);
+        cp_async16(dst + h * 8192 + r * 128 + ((cc ^ (r & 7)) << 4), p.q + ((size_t)bh * p.N + tok) * D + chunk * 8);
       }
+    };
+    auto q_arrive = [&](int is) {
+      if (item_at(p, is) < 0) return;
+      fence_proxy_async_smem();
+      mbar_arrive(&B.q_full[is & 1]);
     };
     // Gates (16 runs of 4 raster tokens per gate array) and the coarse output
     // row of item `is` -> sh.pre[is & 1]; one cp.async group per call on
@@ -674,17 +686,23 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
     };
     load_q(0);
     load_q(1);
+    cp_async_commit();
     prefetch(0);
+    cp_async_wait<1>();
+    q_arrive(0);
+    q_arrive(1);
     for (int is = 0; item_at(p, is) >= 0; ++is) {
       const int item = item_at(p, is);
       const int bh = item / C, ci = item - bh * C;
       const int ct = ci / (Hc * Wc), ch = (ci / Wc) % Hc, cw = ci % Wc;
       const int ob = is & 1;
       // Q of item is + 2 goes into this item's buffer as soon as the item's
-      // S products have completed, not after its O read-out: the 5-D raster
-      // box from HBM then has most of an item to land (waiting for the O
-      // read-out left the S issuer stalled on Q at item boundaries).
-      if (item_at(p, is + 2) >= 0 && (est != 0 || W.wait(&B.q_free[ob], (is >> 1) & 1))) load_q(is + 2);
+      // S products have completed, not after its O read-out, so the copies
+      // from HBM have most of an item to land (waiting for the O read-out
+      // left the S issuer stalled on Q at item boundaries).
+      const bool qnext = item_at(p, is + 2) >= 0 && W.wait(&B.q_free[ob], (is >> 1) & 1);
+      if (qnext) load_q(is + 2);
+      cp_async_commit();
       prefetch(is + 1);
       W.wait(&B.l_full[ob], (is >> 1) & 1);
       const float lsum0 = sh.lpart[ob][0][ra] + sh.lpart[ob][1][ra];
@@ -714,6 +732,7 @@ __global__ void __launch_bounds__(kThreads, 1) fine_attention_kernel(const __gri
       __syncwarp();
       if (lane == 0) mbar_arrive(&B.o_empty);
       cp_async_wait<1>();               // this item's gates and coarse row (older group) landed
+      if (qnext) q_arrive(is + 2);
       if (est == 0) bulk_wait_read0();  // the previous item's output stores have read the staging tile
       epi_sync();
       const Pre& pr = sh.pre[ob];

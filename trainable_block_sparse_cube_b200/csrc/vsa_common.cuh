@@ -54,11 +54,12 @@ struct CoarseParams {
 };
 
 struct FineParams {
-  // tm_q, tm_out: 5-D maps over the raster q and out [BH][T][H][W][D] bf16; a
-  // box is one cube's 4 x 4 x 4 tokens by 64 channels, in the 128-byte swizzle.
+  // tm_out: 5-D map over the raster out [BH][T][H][W][D] bf16; a box is one
+  // cube's 4 x 4 x 4 tokens by 64 channels, in the 128-byte swizzle.
   // tm_k, tm_v: 2-D maps over the cube-major copies (rows of D bf16, 64 x 64 boxes).
-  CUtensorMap tm_q, tm_k, tm_v;
+  CUtensorMap tm_k, tm_v;
   CUtensorMap tm_out;
+  const __nv_bfloat16* q;        // [BH, N, D] raster (query cubes are read from here)
   const int32_t* idx;            // [BH, C, kcap]
   const int32_t* cnt;            // [BH, C] or null (then every row has kcap ids)
   const int32_t* order;          // [BH * C] item order (schedule.cu), or null: items in index order
