@@ -713,26 +713,46 @@ __global__ void __launch_bounds__(128, KIND == 0 ? 2 : 1) coarse_tc_kernel(const
   }
   __syncwarp();
   // Epilogue: warp w holds accumulator rows 32 w .. 32 w + 31 (one per thread).
-  const bool have = mbar_wait(&done, 0, lim);
+  const bool have = __all_sync(0xffffffffu, mbar_wait(&done, 0, lim));  // warp-uniform: the staged path syncs the warp
   if (!have && lane == 0) atomicOr(p.err, kErrTimeout);
   tc_fence_after();
   const int row = m0 + 32 * warp + lane;
+  // Scores: each 32-column group goes through a per-warp [32 rows][36 floats]
+  // staging block in the (now idle) operand stage, so that every warp store
+  // writes four whole 128-byte row segments instead of 16 bytes in each of 32
+  // rows. float4 writes and reads both touch 8 distinct bank groups per
+  // quarter warp (row pitch 9 chunks of 16 bytes).
+  float* stg = reinterpret_cast<float*>(tiles) + warp * 32 * 36;
+  const bool staged = KIND == 0 && (C & 3) == 0;
 #pragma unroll
   for (int cg = 0; cg < S::NT / 32; ++cg) {
     uint32_t r[32];
     tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16) + 32 * cg, r);
     tmem_wait_ld();
+    if (KIND == 0 && staged) {
+      if (!have) continue;
+      __syncwarp();  // the previous group's reads of the block are done
+#pragma unroll
+      for (int e = 0; e < 32; e += 4)
+        *reinterpret_cast<float4*>(stg + lane * 36 + e) =
+            make_float4(__uint_as_float(r[e]) * p.scale, __uint_as_float(r[e + 1]) * p.scale,
+                        __uint_as_float(r[e + 2]) * p.scale, __uint_as_float(r[e + 3]) * p.scale);
+      __syncwarp();
+      const int col = n0 + 32 * cg + 4 * (lane & 7);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int rr = 4 * i + (lane >> 3), grow = m0 + 32 * warp + rr;
+        if (grow < C && col < C)  // C % 4 == 0: a chunk lies wholly inside or outside the row
+          *reinterpret_cast<float4*>(p.s + ((size_t)bh * C + grow) * C + col) =
+              *reinterpret_cast<const float4*>(stg + rr * 36 + 4 * (lane & 7));
+      }
+      continue;
+    }
     if (!have || row >= C) continue;
     if (KIND == 0) {
       float* dst = p.s + ((size_t)bh * C + row) * C + n0 + 32 * cg;
       const int ncol = min(32, C - (n0 + 32 * cg));
-      if ((C & 3) == 0 && ncol == 32) {
-#pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<float4*>(dst + e) =
-              make_float4(__uint_as_float(r[e]) * p.scale, __uint_as_float(r[e + 1]) * p.scale,
-                          __uint_as_float(r[e + 2]) * p.scale, __uint_as_float(r[e + 3]) * p.scale);
-      } else {
+      {
 #pragma unroll
         for (int e = 0; e < 32; ++e)
           if (e < ncol) dst[e] = __uint_as_float(r[e]) * p.scale;
