@@ -30,6 +30,10 @@ SMALL = [
     W["pretrain16k"].with_(name="k_eq_c", heads=1, T=4, H=8, W=12, topk=6),
     W["tiny"].with_(name="single_cube", T=4, H=4, W=4, heads=2, topk=1),
     W["large77k"].with_(name="sin_k40_c80", heads=2, T=8, H=16, W=40, topk=40),
+    # odd cube counts (the select kernel's unpaired score loads); 243 cubes put
+    # 65..256 keys above the lane-maxima bound (its wider candidate sets)
+    W["pretrain16k"].with_(name="odd_c27_k5", heads=2, T=12, H=12, W=12, topk=5),
+    W["pretrain16k"].with_(name="odd_c243_k32", heads=1, T=36, H=36, W=12, topk=32),
 ]
 
 
