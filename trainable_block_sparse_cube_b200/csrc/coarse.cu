@@ -153,12 +153,38 @@ __device__ __forceinline__ void load_row_regs(const CoarseParams& p, int row, in
   }
 }
 
+// The probabilities v * inv_l of a register-resident row (load_row_regs
+// layout) as TERMS bf16 terms (hi, mid[, lo]), written as bf16 pairs.
+template <int TERMS>
+__device__ __forceinline__ void store_p_terms(const CoarseParams& p, int row, int lane, const float (&v)[32],
+                                              float inv_l) {
+  const size_t plane = (size_t)p.BH * p.C * p.Cp;
+  __nv_bfloat16* prow = p.psplit + (size_t)row * p.Cp;
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    const int j = 64 * u + 2 * lane;
+    if (j < p.Cp) {  // Cp is a multiple of 8: the pair j, j + 1 lies inside the row
+      float x0 = v[2 * u] * inv_l, x1 = v[2 * u + 1] * inv_l;
+#pragma unroll
+      for (int t = 0; t < TERMS; ++t) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+        *reinterpret_cast<__nv_bfloat162*>(prow + t * plane + j) = h;
+        if (t + 1 < TERMS) {
+          const float2 back = __bfloat1622float2(h);
+          x0 -= back.x;
+          x1 -= back.y;
+        }
+      }
+    }
+  }
+}
+
 // Softmax of a register-resident row (load_row_regs layout) with row max lm:
 // writes the probabilities' terms as bf16 pairs, returns the row max in log2
 // units (mb) and the row sum l. v is overwritten with the numerators.
+template <bool SPLIT_TERMS>
 __device__ __forceinline__ void softmax_store_regs(const CoarseParams& p, int row, int lane, float (&v)[32], float lm,
                                                    float& mb, float& l) {
-  const int C = p.C;
   mb = warp_max(lm) * kLog2e;
   float ls = 0.f;
 #pragma unroll
@@ -168,21 +194,26 @@ __device__ __forceinline__ void softmax_store_regs(const CoarseParams& p, int ro
   }
   l = warp_sum(ls);
   const float inv_l = 1.0f / l;
-  const size_t plane = (size_t)p.BH * C * p.Cp;
-  __nv_bfloat16* prow = p.psplit + (size_t)row * p.Cp;
-  const int terms = p.p_terms;
+  if (SPLIT_TERMS) {  // one copy of the store loop per term count: no wasted third term in the forward
+    if (p.p_terms > 2) store_p_terms<3>(p, row, lane, v, inv_l);
+    else store_p_terms<2>(p, row, lane, v, inv_l);
+  } else {  // one loop for either count (fewer registers)
+    const size_t plane = (size_t)p.BH * p.C * p.Cp;
+    __nv_bfloat16* prow = p.psplit + (size_t)row * p.Cp;
+    const int terms = p.p_terms;
 #pragma unroll
-  for (int u = 0; u < 16; ++u) {
-    const int j = 64 * u + 2 * lane;
-    if (j < p.Cp) {  // Cp is a multiple of 8: the pair j, j + 1 lies inside the row
-      float x0 = v[2 * u] * inv_l, x1 = v[2 * u + 1] * inv_l;
+    for (int u = 0; u < 16; ++u) {
+      const int j = 64 * u + 2 * lane;
+      if (j < p.Cp) {
+        float x0 = v[2 * u] * inv_l, x1 = v[2 * u + 1] * inv_l;
 #pragma unroll
-      for (int t = 0; t < 3; ++t) {
-        const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
-        const float2 back = __bfloat1622float2(h);
-        x0 -= back.x;
-        x1 -= back.y;
-        if (t < terms) *reinterpret_cast<__nv_bfloat162*>(prow + t * plane + j) = h;
+        for (int t = 0; t < 3; ++t) {
+          const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+          const float2 back = __bfloat1622float2(h);
+          x0 -= back.x;
+          x1 -= back.y;
+          if (t < terms) *reinterpret_cast<__nv_bfloat162*>(prow + t * plane + j) = h;
+        }
       }
     }
   }
@@ -210,7 +241,7 @@ __device__ __forceinline__ void row_softmax_regs(const CoarseParams& p, int row,
         lm = fmaxf(lm, v[2 * u + h]);
       }
   }
-  softmax_store_regs(p, row, lane, v, lm, mb, l);
+  softmax_store_regs<false>(p, row, lane, v, lm, mb, l);
   __syncwarp();
 }
 
@@ -403,7 +434,7 @@ __device__ __forceinline__ void select_topk_regs(const CoarseParams& p, int row,
 #pragma unroll
   for (int e = 0; e < 32; ++e) v[e] = key_value(__float_as_uint(v[e]));
   float mb, l;
-  softmax_store_regs(p, row, lane, v, key_value(hi), mb, l);
+  softmax_store_regs<true>(p, row, lane, v, key_value(hi), mb, l);
   __syncwarp();
   int32_t* irow = p.idx + (size_t)row * p.kcap;
   if (n <= 32) topk_bitmap_emit<1>(keys, cidx, n, Kt, lo, hi, bm, irow);
