@@ -286,8 +286,8 @@ vsa_status vsa_set_debug_stall(vsa_plan_t plan, int on);
  * "Faster Video Diffusion with Trainable Sparse Attention", "Approach": one
  * cube of 4 x 4 x 4 tokens is one tile). Every run writes the cube-major
  * copies of k and v (regions k_cube, v_cube), which the fine-attention kernel
- * streams; it reads q straight from the raster tensor with 5-D TMA boxes, so
- * q's copy is not needed. When `on` is nonzero, later runs of this plan also
+ * streams; it reads q straight from the raster tensor (16-byte copies of each
+ * query cube's token rows), so q's copy is not needed. When `on` is nonzero, later runs of this plan also
  * write q's copy into region q_cube (one extra write of q); off by default. */
 vsa_status vsa_set_cube_major_copies(vsa_plan_t plan, int on);
 

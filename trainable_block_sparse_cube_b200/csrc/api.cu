@@ -207,7 +207,7 @@ vsa_status encode_coarse_maps(vsa_plan_s* P) {
   return e;
 }
 
-// 5-D map over a raster tensor [BH][T][H][W][D] bf16 (q or out): a box
+// 5-D map over a raster output [BH][T][H][W][D] bf16 (out, dq, dk, dv): a box
 // is one cube's 4 x 4 x 4 tokens by 64 channels, laid out in shared memory as
 // 64 rows (in-cube slot order) of 128 bytes in the 128-byte swizzle.
 vsa_status encode_raster_map(CUtensorMap* m, const void* base, const vsa_config& c, int BH) {
