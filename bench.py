@@ -95,6 +95,21 @@ def fine_source_sha():
     return h.hexdigest()
 
 
+# An M=64 tcgen05 MMA runs at half the M=128 rate: 4,096 bf16 FLOP per cycle per SM
+# (an M=64 N=128 K=16 product takes 64 cycles, measured), so a query-cube tile
+# (64 tokens) caps the fine kernel at this rate whatever the schedule.
+M64_FLOP_PER_CYCLE_PER_SM = 4096.0
+
+
+def m64_rate_tflops(device, sm_mhz):
+    """The M=64 MMA rate of the whole GPU at the sampled SM clock (TFLOP/s), or None."""
+    try:
+        sms = torch.cuda.get_device_properties(device).multi_processor_count
+        return sms * M64_FLOP_PER_CYCLE_PER_SM * float(sm_mhz) * 1e6 / 1e12
+    except Exception:
+        return None
+
+
 def fine_traffic():
     """DRAM bytes per launch of the fine kernel from the committed ncu record
     (profiles/*.json), if it was captured on the current kernel source; else None."""
@@ -516,6 +531,7 @@ def rank_main(args):
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     g_bytes = gather_bytes(wl)
     kv_l2_gbs = f_fine / FINE_FLOP_PER_L2_BYTE / (fine_ms * 1e-3) / 1e9
+    m64_rate = m64_rate_tflops(out.device, (clocks or {}).get("sm_mhz"))
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": med_max, "ms_per_step_mean": t_max / args.steps,
@@ -528,6 +544,8 @@ def rank_main(args):
                      "peak_source": f"{peak_src} bf16_tflops (burst)",
                      "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
                      "frac_of_datasheet_2250": achieved / 2250.0,
+                     "frac_of_m64_rate": (achieved / m64_rate) if m64_rate else None,
+                     "m64_rate": m64_rate,
                      "stage_timing": f"median over the {args.steps} timed calls (stage events in the same stream)"},
         "l2_roofline": {"kv_bytes_per_s_gbs": kv_l2_gbs, "l2_read_gbs_measured": l2_gbs,
                         "frac": kv_l2_gbs / l2_gbs if l2_gbs else None,
